@@ -1,0 +1,356 @@
+"""Benchmark of the importance-sampled block-sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan14_10]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed on host cores
+
+One step = the whole hot path on one attention layer: isa_score -> isa_select
+-> isa_attention, inputs resident in HBM.  Prints one JSON line (rank 0).
+
+value        computed TFLOP/s of the step: the attention FLOPs the plan makes
+             the kernel compute (4 d per query row per selected valid key row,
+             padding excluded) divided by the step time.
+ms_per_step  milliseconds per call of the whole path.
+roofline     the attention kernel (dominant): computed FLOPs per launch / its
+             event-timed duration, against the measured bf16 tensor peak.
+e2e          the same metric through isa_pipeline_host: pinned host Q/K/V in,
+             host O out, copies inside the timed region.
+Multi-GPU: one process per GPU (torchrun); every rank runs its own layer
+(weak scaling, no data-path collective); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse IS-attention ms/call + computed TFLOP/s vs B200 BF16 peak, per shape"
+UNIT = "TFLOP/s (computed)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def plan_flops(idx: np.ndarray, offsets: np.ndarray, N: int, Bk: int, d: int) -> float:
+    """Computed attention FLOPs of a plan: 4 d per (query row, selected valid key row)."""
+    L = np.minimum(Bk, N - np.arange(-(-N // Bk)) * Bk)           # valid rows of each key block
+    keys = L[idx].sum(axis=-1).astype(np.float64)                   # [B, H, G]
+    rows = np.diff(offsets).astype(np.float64)                      # [G]
+    return float(4.0 * d * (keys * rows[None, None, :]).sum())
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_query_id(dev) -> str:
+    """nvidia-smi id of the torch device (its UUID when torch exposes it)."""
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        if u:
+            return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        pass
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    if vis:
+        return vis.split(",")[dev.index or 0]
+    return str(dev.index or 0)
+
+
+def cpu_oracle_sample(w, inp, target_s: float = 12.0):
+    """Time the oracle (score -> select -> attention) on the first groups of
+    head 0, growing the sample until it takes about `target_s` seconds."""
+    import oracle
+    from block_sparse_importance_b200 import workloads as wl
+    q = wl.bf16_bits(inp.q[:, :1])
+    k = wl.bf16_bits(inp.k[:, :1])
+    v = wl.bf16_bits(inp.v[:, :1])
+    off = inp.offsets
+    G = len(off) - 1
+    N, d = q.shape[2], q.shape[3]
+
+    def run(n_groups):
+        sub = off[:n_groups + 1]
+        t0 = time.perf_counter()
+        mass, _, _, _ = oracle.score(q, k, sub, w.k_block, w.n_clusters, w.n_iters, w.scale)
+        idx, lw, _ = oracle.select(mass.astype(np.float32), w.n_exact, w.n_sample, w.seed)
+        oracle.attention(q, k, v, sub, w.k_block, idx, lw, w.scale, [(0, 0, g) for g in range(n_groups)])
+        dt = time.perf_counter() - t0
+        return dt, plan_flops(idx, sub, N, w.k_block, d)
+
+    n = min(G, 2)
+    dt, fl = run(n)
+    while dt < target_s / 4 and n < G:
+        n = min(G, max(n + 1, int(n * min(8.0, target_s / max(dt, 1e-3)))))
+        dt, fl = run(n)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "head 0, first %d of %d query groups of %s: oracle score+select+attention (fp64), %.1f s"
+                      % (n, G, w.name, dt)}
+
+
+def reference_arm(args):
+    """--impl reference: the fp64 oracle on the host cores, bounded samples."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from block_sparse_importance_b200 import workloads as wl
+    w = wl.preset(args.workload)
+    inp = wl.make_inputs(w, "cpu", heads=1)
+    vals = []
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, inp, target_s=2.0)
+    for _ in range(args.steps):
+        vals.append(cpu_oracle_sample(w, inp, target_s=args.ref_seconds))
+    v = statistics.median(x["value"] for x in vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": vals[-1]["cores"], "kind": "oracle",
+                             "sample": vals[-1]["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w):
+    return {"workload": w.name, "heads": w.heads, "head_dim": w.head_dim, "seq_len": w.seq_len,
+            "grid": list(w.grid), "q_block": w.q_block, "k_block": w.k_block, "n_exact": w.n_exact,
+            "n_sample": w.n_sample, "n_clusters": w.n_clusters, "n_iters": w.n_iters,
+            "density": round(w.density, 4), "variable_groups": w.variable_groups, "batch": w.batch,
+            "l2": "inputs larger than L2 (no flush)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="wan14_10")
+    ap.add_argument("--impl", default="isa", choices=["isa", "reference"])
+    ap.add_argument("--ref-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    import torch.distributed as dist
+    from block_sparse_importance_b200 import isa
+    from block_sparse_importance_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    w = wl.preset(args.workload, seed=0)
+    inp = wl.make_inputs(w, str(dev))
+    q, k, v = inp.q, inp.k, inp.v
+    off_dev = torch.from_numpy(inp.offsets).to(dev) if w.variable_groups else None
+    lay = isa.layout_for(q, w.k_block, w.q_block, q_offsets=off_dev, scale=w.scale)
+    ctx = isa.context(local)
+    stream = torch.cuda.current_stream()
+    B, H, N, d = q.shape
+    G, nK, S = lay.num_groups, lay.n_key_blocks, w.n_select
+    mass = torch.empty(B, H, G, nK, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, H, G, S, dtype=torch.int32, device=dev)
+    lw = torch.empty(B, H, G, S, dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    sws = torch.empty(isa.score_workspace_bytes(lay, w.n_clusters) + 256, dtype=torch.uint8, device=dev)
+    aws_n = isa.attention_workspace_bytes(lay)
+    aws = torch.empty(aws_n + 256, dtype=torch.uint8, device=dev) if aws_n else None
+
+    def step(ev=None):
+        isa.score(q, k, lay, w.n_clusters, w.n_iters, mass=mass, workspace=sws, ctx=ctx)
+        isa.select(mass, lay, w.n_exact, w.n_sample, w.seed, idx=idx, log_w=lw, ctx=ctx)
+        if ev is not None:
+            ev[0].record(stream)
+        isa.attention(q, k, v, idx, lw, lay, out=out, workspace=aws, ctx=ctx)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = ctx.sync_status()
+    if st != isa.ISA_OK:
+        raise RuntimeError("device status after warm-up: %s" % isa.status_string(st))
+    flops = plan_flops(idx.cpu().numpy(), inp.offsets, N, w.k_block, d)   # per step (per rank)
+
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_query_id(dev)) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(attn_ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    clocks = clk.summary()
+    st = ctx.sync_status()
+    if st != isa.ISA_OK:
+        raise RuntimeError("device status after timing: %s" % isa.status_string(st))
+    elapsed_ms = t0.elapsed_time(t1)
+    attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / args.steps
+    if world > 1:
+        tt = torch.tensor([elapsed_ms, attn_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms, attn_ms = float(tt[0]), float(tt[1])
+    ms_step = elapsed_ms / args.steps
+    value = world * flops / (ms_step * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "kernel": "attn_kernel<128>",
+                "peak_source": "%s bf16_tflops_sustained (kernel timed inside a multi-kernel step loop)" % peak_src}
+
+    # dense limit, same tensors (context for the speedup analogue)
+    dense_ms = None
+    if rank == 0:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        isa.dense_attention(q, k, v, lay, out=out, ctx=ctx)
+        e0.record(stream)
+        for _ in range(2):
+            isa.dense_attention(q, k, v, lay, out=out, ctx=ctx)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = e0.elapsed_time(e1) / 2
+
+    # end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        p = isa.params(w.n_clusters, w.n_iters, w.n_exact, w.n_sample, w.seed)
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        oh = torch.empty_like(qh).pin_memory()
+        del sws
+        arena = torch.empty(isa.pipeline_host_workspace_bytes(lay, p) + 256, dtype=torch.uint8, device=dev)
+        for _ in range(2):
+            isa.pipeline_host(qh, kh, vh, oh, lay, p, arena, ctx=ctx, device=local)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(2, min(args.steps, 5))
+        e0.record(stream)
+        for _ in range(n_e2e):
+            isa.pipeline_host(qh, kh, vh, oh, lay, p, arena, ctx=ctx, device=local)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt[0])
+        nbytes = q.numel() * q.element_size()
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+               "api": "isa_pipeline_host (pinned host buffers)"}
+        del arena
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = wl.make_inputs(w, "cpu", heads=1)
+        cpu = cpu_oracle_sample(w, inp_cpu, target_s=args.ref_seconds)
+
+    launches_per_step = 5 + (1 if aws_n else 0)
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w),
+                "attention_ms": attn_ms, "attention_tflops": achieved,
+                "dense_equiv_tflops": world * 4.0 * d * N * N * H * B / (attn_ms * 1e-3) / 1e12,
+                "dense_attention_ms": dense_ms,
+                "sparse_vs_dense": (dense_ms / attn_ms) if dense_ms else None,
+                "computed_tflop_per_step": flops / 1e12,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,422 @@
+// C ABI of libisa.so (declared in include/isa.h): argument checks, the
+// per-context device status word, workspace carving and kernel launches.
+// The library allocates nothing in a call path; every device buffer belongs
+// to the caller.
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "isa.h"
+#include "isa_internal.h"
+
+struct isa_context {
+  int device;
+  int num_sms;
+  int* d_status;
+  char last_error[512];
+};
+
+namespace {
+
+using namespace isa_impl;
+
+isa_status fail(isa_context* ctx, isa_status s, const char* fmt, ...) {
+  if (ctx) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(ctx->last_error, sizeof(ctx->last_error), fmt, ap);
+    va_end(ap);
+  }
+  return s;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Makes the context's device current for the duration of a call.
+class DeviceGuard {
+ public:
+  explicit DeviceGuard(int dev) {
+    ok_ = cudaGetDevice(&prev_) == cudaSuccess;
+    if (ok_ && prev_ != dev) ok_ = cudaSetDevice(dev) == cudaSuccess;
+    restore_ = ok_ && prev_ != dev;
+  }
+  ~DeviceGuard() {
+    if (restore_) cudaSetDevice(prev_);
+  }
+  bool ok() const { return ok_; }
+
+ private:
+  int prev_ = 0;
+  bool ok_ = false, restore_ = false;
+};
+
+int nblocks(const isa_shape* s) { return (s->seq_len + s->k_block - 1) / s->k_block; }
+
+isa_status check_shape(isa_context* ctx, const isa_shape* s) {
+  if (!ctx) return ISA_ERR_INVALID_ARG;
+  ctx->last_error[0] = 0;
+  if (!s) return fail(ctx, ISA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->batch < 1 || s->heads < 1 || s->seq_len < 1)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "batch, heads and seq_len must be >= 1");
+  if (s->head_dim != 64 && s->head_dim != 128)
+    return fail(ctx, ISA_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are built", s->head_dim);
+  if (s->k_block != 16 && s->k_block != 32 && s->k_block != 64 && s->k_block != 128)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "k_block %d: must be 16, 32, 64 or 128", s->k_block);
+  if (s->num_groups < 1) return fail(ctx, ISA_ERR_INVALID_ARG, "num_groups must be >= 1");
+  if (!s->q_offsets) {
+    if (s->q_block < 1) return fail(ctx, ISA_ERR_INVALID_ARG, "q_block must be >= 1");
+    const long long g = (static_cast<long long>(s->seq_len) + s->q_block - 1) / s->q_block;
+    if (g != s->num_groups)
+      return fail(ctx, ISA_ERR_INVALID_ARG, "num_groups %d != ceil(seq_len / q_block) = %lld", s->num_groups, g);
+  } else {
+    if (!aligned(s->q_offsets, 4)) return fail(ctx, ISA_ERR_INVALID_ARG, "q_offsets not 4-byte aligned");
+    if (s->num_groups > s->seq_len) return fail(ctx, ISA_ERR_INVALID_ARG, "more groups than rows");
+  }
+  if (!std::isfinite(s->scale)) return fail(ctx, ISA_ERR_INVALID_ARG, "scale must be finite");
+  const long long bh = static_cast<long long>(s->batch) * s->heads;
+  if (bh * s->seq_len > (1LL << 40) || bh > (1LL << 30))
+    return fail(ctx, ISA_ERR_INVALID_ARG, "tensor too large");
+  return ISA_OK;
+}
+
+isa_status check_ptr(isa_context* ctx, const void* p, const char* name, size_t align) {
+  if (!p) return fail(ctx, ISA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, align)) return fail(ctx, ISA_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+  return ISA_OK;
+}
+
+isa_status cuda_status(isa_context* ctx, int e, const char* what) {
+  if (e == 0) return ISA_OK;
+  if (e < 0) return fail(ctx, ISA_ERR_CUDA, "%s: tensor map encoding failed", what);
+  return fail(ctx, ISA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(static_cast<cudaError_t>(e)));
+}
+
+#define ISA_TRY(x)                  \
+  do {                              \
+    const isa_status s_ = (x);      \
+    if (s_ != ISA_OK) return s_;    \
+  } while (0)
+
+size_t attn_ws_bytes(const isa_shape* s) {
+  const bool list = s->q_offsets != nullptr || s->q_block > 128;
+  return list ? round_up(attn_list_workspace_bytes(s->seq_len, s->num_groups)) : 0;
+}
+
+isa_status do_score(isa_context* ctx, const isa_shape* s, const void* q, const void* k, int32_t C, int32_t iters,
+                    float* mass, float* centroids, int32_t* counts, void* ws, size_t ws_bytes, cudaStream_t st) {
+  ISA_TRY(check_ptr(ctx, q, "q", 16));
+  ISA_TRY(check_ptr(ctx, k, "k", 16));
+  ISA_TRY(check_ptr(ctx, mass, "mass", 16));
+  if (C < 1 || C > 16) return fail(ctx, ISA_ERR_INVALID_ARG, "n_clusters %d: must be 1..16", C);
+  if (iters < 1 || iters > 16) return fail(ctx, ISA_ERR_INVALID_ARG, "n_iters %d: must be 1..16", iters);
+  if (centroids && !aligned(centroids, 16)) return fail(ctx, ISA_ERR_INVALID_ARG, "centroids not 16-byte aligned");
+  if (counts && !aligned(counts, 4)) return fail(ctx, ISA_ERR_INVALID_ARG, "counts not 4-byte aligned");
+  const size_t need = score_workspace_bytes(s->batch, s->heads, s->seq_len, s->head_dim, s->num_groups, s->k_block, C);
+  if (!ws || ws_bytes < need)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "score workspace %zu bytes < %zu needed", ws_bytes, need);
+  if (!aligned(ws, 256)) return fail(ctx, ISA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  const size_t BH = static_cast<size_t>(s->batch) * s->heads;
+  const size_t nK = nblocks(s);
+  char* w = static_cast<char*>(ws);
+  ScoreLaunch l{};
+  l.B = s->batch;
+  l.H = s->heads;
+  l.N = s->seq_len;
+  l.D = s->head_dim;
+  l.G = s->num_groups;
+  l.Bk = s->k_block;
+  l.q_block = s->q_block;
+  l.C = C;
+  l.iters = iters;
+  l.q_offsets = s->q_offsets;
+  l.scale = s->scale;
+  l.q = q;
+  l.k = k;
+  l.mass = mass;
+  l.kbar = reinterpret_cast<float*>(w);
+  w += round_up(BH * nK * s->head_dim * 4);
+  l.centroids = centroids ? centroids : reinterpret_cast<float*>(w);
+  w += round_up(BH * s->num_groups * C * s->head_dim * 4);
+  l.counts = counts ? counts : reinterpret_cast<int32_t*>(w);
+  l.status = ctx->d_status;
+  l.num_sms = ctx->num_sms;
+  return cuda_status(ctx, launch_score(l, st), "isa_score");
+}
+
+isa_status do_select(isa_context* ctx, const isa_shape* s, const float* mass, int32_t ne, int32_t ns, uint64_t seed,
+                     int32_t* idx, float* log_w, cudaStream_t st) {
+  ISA_TRY(check_ptr(ctx, mass, "mass", 4));
+  ISA_TRY(check_ptr(ctx, idx, "idx", 4));
+  ISA_TRY(check_ptr(ctx, log_w, "log_w", 4));
+  const int nK = nblocks(s);
+  if (ne < 0 || ns < 0 || ne + ns < 1 || ne + ns > nK)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "need 0 <= n_exact, n_sample and 1 <= n_exact + n_sample <= nK = %d", nK);
+  if (nK > 16384) return fail(ctx, ISA_ERR_UNSUPPORTED, "nK = %d key blocks: at most 16384 are built", nK);
+  SelectLaunch l{};
+  l.B = s->batch;
+  l.H = s->heads;
+  l.G = s->num_groups;
+  l.nK = nK;
+  l.n_exact = ne;
+  l.n_sample = ns;
+  l.seed = seed;
+  l.mass = mass;
+  l.idx = idx;
+  l.log_w = log_w;
+  l.status = ctx->d_status;
+  return cuda_status(ctx, launch_select(l, st), "isa_select");
+}
+
+isa_status do_attention(isa_context* ctx, const isa_shape* s, const void* q, const void* k, const void* v,
+                        const int32_t* idx, const float* log_w, int32_t n_sel, void* out, float* lse, void* ws,
+                        size_t ws_bytes, bool dense, cudaStream_t st) {
+  ISA_TRY(check_ptr(ctx, q, "q", 16));
+  ISA_TRY(check_ptr(ctx, k, "k", 16));
+  ISA_TRY(check_ptr(ctx, v, "v", 16));
+  ISA_TRY(check_ptr(ctx, out, "out", 16));
+  if (lse && !aligned(lse, 4)) return fail(ctx, ISA_ERR_INVALID_ARG, "lse not 4-byte aligned");
+  AttnLaunch l{};
+  l.B = s->batch;
+  l.H = s->heads;
+  l.N = s->seq_len;
+  l.D = s->head_dim;
+  l.G = s->num_groups;
+  l.Bk = s->k_block;
+  l.q_block = s->q_block;
+  l.q_offsets = s->q_offsets;
+  l.out = out;
+  l.lse = lse;
+  l.scale = s->scale;
+  l.status = ctx->d_status;
+  l.num_sms = ctx->num_sms;
+  if (dense) {
+    l.mode = kAttnDense;
+    l.S = 1;
+    l.G = 1;
+  } else {
+    ISA_TRY(check_ptr(ctx, idx, "idx", 4));
+    ISA_TRY(check_ptr(ctx, log_w, "log_w", 4));
+    if (n_sel < 1) return fail(ctx, ISA_ERR_INVALID_ARG, "n_sel must be >= 1");
+    l.S = n_sel;
+    l.idx = idx;
+    l.log_w = log_w;
+    const size_t need = attn_ws_bytes(s);
+    if (need) {
+      if (!ws || ws_bytes < need)
+        return fail(ctx, ISA_ERR_INVALID_ARG, "attention workspace %zu bytes < %zu needed", ws_bytes, need);
+      if (!aligned(ws, 16)) return fail(ctx, ISA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+      l.mode = kAttnList;
+      l.workspace = ws;
+    } else {
+      l.mode = kAttnGroups;
+    }
+  }
+  return cuda_status(ctx, launch_attention(l, q, k, v, st), dense ? "isa_dense_attention" : "isa_attention");
+}
+
+size_t pipeline_bytes(const isa_shape* s, const isa_params* p) {
+  const size_t rows = static_cast<size_t>(s->batch) * s->heads * s->num_groups;
+  const size_t S = static_cast<size_t>(p->n_exact) + p->n_sample;
+  return round_up(score_workspace_bytes(s->batch, s->heads, s->seq_len, s->head_dim, s->num_groups, s->k_block,
+                                        p->n_clusters)) +
+         round_up(rows * nblocks(s) * 4) + 2 * round_up(rows * S * 4) + attn_ws_bytes(s);
+}
+
+isa_status do_pipeline(isa_context* ctx, const isa_shape* s, const isa_params* p, const void* q, const void* k,
+                       const void* v, void* out, float* lse, int32_t* plan_idx, float* plan_lw, void* ws,
+                       size_t ws_bytes, cudaStream_t st) {
+  if (!p) return fail(ctx, ISA_ERR_INVALID_ARG, "params is NULL");
+  if (p->n_clusters < 1 || p->n_clusters > 16) return fail(ctx, ISA_ERR_INVALID_ARG, "n_clusters must be 1..16");
+  const size_t need = pipeline_bytes(s, p);
+  if (!ws || ws_bytes < need)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "pipeline workspace %zu bytes < %zu needed", ws_bytes, need);
+  if (!aligned(ws, 256)) return fail(ctx, ISA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  const size_t rows = static_cast<size_t>(s->batch) * s->heads * s->num_groups;
+  const size_t S = static_cast<size_t>(p->n_exact) + p->n_sample;
+  char* w = static_cast<char*>(ws);
+  const size_t score_ws = round_up(score_workspace_bytes(s->batch, s->heads, s->seq_len, s->head_dim, s->num_groups,
+                                                         s->k_block, p->n_clusters));
+  void* sws = w;
+  w += score_ws;
+  float* mass = reinterpret_cast<float*>(w);
+  w += round_up(rows * nblocks(s) * 4);
+  int32_t* idx = plan_idx ? plan_idx : reinterpret_cast<int32_t*>(w);
+  w += round_up(rows * S * 4);
+  float* lw = plan_lw ? plan_lw : reinterpret_cast<float*>(w);
+  w += round_up(rows * S * 4);
+  void* aws = w;
+  ISA_TRY(do_score(ctx, s, q, k, p->n_clusters, p->n_iters, mass, nullptr, nullptr, sws, score_ws, st));
+  ISA_TRY(do_select(ctx, s, mass, p->n_exact, p->n_sample, p->seed, idx, lw, st));
+  return do_attention(ctx, s, q, k, v, idx, lw, static_cast<int32_t>(S), out, lse, aws, attn_ws_bytes(s), false, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+isa_status isa_create(int device, isa_context** out) {
+  if (!out) return ISA_ERR_INVALID_ARG;
+  *out = nullptr;
+  int prev = 0;
+  if (cudaGetDevice(&prev) != cudaSuccess) return ISA_ERR_CUDA;
+  if (cudaSetDevice(device) != cudaSuccess) return ISA_ERR_CUDA;
+  cudaDeviceProp prop;
+  isa_status st = ISA_OK;
+  int* d_status = nullptr;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) {
+    st = ISA_ERR_CUDA;
+  } else if (prop.major != 10 || prop.minor != 0) {
+    st = ISA_ERR_UNSUPPORTED;  // the kernels are built for sm_100a only
+  } else if (cudaMalloc(&d_status, sizeof(int)) != cudaSuccess || cudaMemset(d_status, 0, sizeof(int)) != cudaSuccess) {
+    st = ISA_ERR_CUDA;
+  }
+  if (st == ISA_OK) {
+    isa_context* c = new isa_context();
+    c->device = device;
+    c->num_sms = prop.multiProcessorCount;
+    c->d_status = d_status;
+    c->last_error[0] = 0;
+    *out = c;
+  } else if (d_status) {
+    cudaFree(d_status);
+  }
+  cudaSetDevice(prev);
+  return st;
+}
+
+void isa_destroy(isa_context* ctx) {
+  if (!ctx) return;
+  DeviceGuard g(ctx->device);
+  cudaFree(ctx->d_status);
+  delete ctx;
+}
+
+const char* isa_status_string(isa_status s) {
+  switch (s) {
+    case ISA_OK: return "ok";
+    case ISA_ERR_INVALID_ARG: return "invalid argument";
+    case ISA_ERR_UNSUPPORTED: return "unsupported";
+    case ISA_ERR_CUDA: return "CUDA error";
+    case ISA_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case ISA_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+const char* isa_last_error(const isa_context* ctx) { return ctx ? ctx->last_error : "no context"; }
+
+isa_status isa_sync_status(isa_context* ctx, void* stream) {
+  if (!ctx) return ISA_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, ctx->d_status, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->d_status, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(ctx, ISA_ERR_CUDA, "isa_sync_status: %s", cudaGetErrorString(e));
+  if (h == ISA_ERR_TIMEOUT) return ISA_ERR_TIMEOUT;
+  if (h != 0) return ISA_ERR_DEVICE_CHECK;
+  return ISA_OK;
+}
+
+size_t isa_score_workspace_bytes(const isa_shape* s, int32_t n_clusters) {
+  if (!s || n_clusters < 1) return 0;
+  return score_workspace_bytes(s->batch, s->heads, s->seq_len, s->head_dim, s->num_groups, s->k_block, n_clusters);
+}
+
+isa_status isa_score(isa_context* ctx, const isa_shape* shape, const void* q, const void* k, int32_t n_clusters,
+                     int32_t n_iters, float* mass, float* centroids, int32_t* counts, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  return do_score(ctx, shape, q, k, n_clusters, n_iters, mass, centroids, counts, workspace, workspace_bytes,
+                  static_cast<cudaStream_t>(stream));
+}
+
+isa_status isa_select(isa_context* ctx, const isa_shape* shape, const float* mass, int32_t n_exact, int32_t n_sample,
+                      uint64_t seed, int32_t* idx, float* log_w, void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  return do_select(ctx, shape, mass, n_exact, n_sample, seed, idx, log_w, static_cast<cudaStream_t>(stream));
+}
+
+size_t isa_attention_workspace_bytes(const isa_shape* s) { return s ? attn_ws_bytes(s) : 0; }
+
+isa_status isa_attention(isa_context* ctx, const isa_shape* shape, const void* q, const void* k, const void* v,
+                         const int32_t* idx, const float* log_w, int32_t n_sel, void* out, float* lse,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  return do_attention(ctx, shape, q, k, v, idx, log_w, n_sel, out, lse, workspace, workspace_bytes, false,
+                      static_cast<cudaStream_t>(stream));
+}
+
+isa_status isa_dense_attention(isa_context* ctx, const isa_shape* shape, const void* q, const void* k,
+                               const void* v, void* out, float* lse, void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  return do_attention(ctx, shape, q, k, v, nullptr, nullptr, 0, out, lse, nullptr, 0, true,
+                      static_cast<cudaStream_t>(stream));
+}
+
+size_t isa_pipeline_workspace_bytes(const isa_shape* s, const isa_params* p) {
+  if (!s || !p || p->n_clusters < 1) return 0;
+  return pipeline_bytes(s, p);
+}
+
+isa_status isa_pipeline(isa_context* ctx, const isa_shape* shape, const isa_params* params, const void* q,
+                        const void* k, const void* v, void* out, float* lse, int32_t* plan_idx, float* plan_log_w,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  return do_pipeline(ctx, shape, params, q, k, v, out, lse, plan_idx, plan_log_w, workspace, workspace_bytes,
+                     static_cast<cudaStream_t>(stream));
+}
+
+size_t isa_pipeline_host_workspace_bytes(const isa_shape* s, const isa_params* p) {
+  if (!s || !p || p->n_clusters < 1) return 0;
+  const size_t t = round_up(static_cast<size_t>(s->batch) * s->heads * s->seq_len * s->head_dim * 2);
+  return 4 * t + pipeline_bytes(s, p);
+}
+
+isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, const isa_params* params, const void* q_host,
+                             const void* k_host, const void* v_host, void* out_host, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  if (!params) return fail(ctx, ISA_ERR_INVALID_ARG, "params is NULL");
+  if (!q_host || !k_host || !v_host || !out_host) return fail(ctx, ISA_ERR_INVALID_ARG, "host buffer is NULL");
+  const size_t need = isa_pipeline_host_workspace_bytes(shape, params);
+  if (!workspace || workspace_bytes < need)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "host-pipeline arena %zu bytes < %zu needed", workspace_bytes, need);
+  if (!aligned(workspace, 256)) return fail(ctx, ISA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(shape->batch) * shape->heads * shape->seq_len * shape->head_dim * 2;
+  const size_t t = round_up(bytes);
+  char* w = static_cast<char*>(workspace);
+  void *dq = w, *dk = w + t, *dv = w + 2 * t, *dout = w + 3 * t;
+  cudaError_t e = cudaMemcpyAsync(dq, q_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host copy in: %s", cudaGetErrorString(e));
+  ISA_TRY(do_pipeline(ctx, shape, params, dq, dk, dv, dout, nullptr, nullptr, nullptr, w + 4 * t, need - 4 * t, st));
+  e = cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host copy out: %s", cudaGetErrorString(e));
+  return ISA_OK;
+}
+
+}  // extern "C"

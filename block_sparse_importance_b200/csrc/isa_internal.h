@@ -1,0 +1,74 @@
+// Internal launch interface between the C-ABI layer (isa_api.cu) and the
+// kernels.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace isa_impl {
+
+// Device status codes (same values as isa_status).
+enum : int { kStatusOk = 0, kStatusTimeout = 4, kStatusDeviceCheck = 5 };
+
+// Per-wait time limit of every bounded pipeline wait in the kernels.
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+
+// ------------------------------------------------------------- attention
+enum AttnMode : int {
+  kAttnGroups = 0,  // uniform query groups of <= 128 rows: one tile per group
+  kAttnList = 1,    // tile list built on the device (clusters or groups > 128 rows)
+  kAttnDense = 2    // all keys, no plan
+};
+
+struct AttnLaunch {
+  int B, H, N, D, G, S, Bk, q_block;
+  int mode;
+  const int32_t* q_offsets;  // kAttnList: device [G+1] (NULL: uniform q_block groups)
+  const int32_t* idx;
+  const float* log_w;
+  void* out;
+  float* lse;
+  void* workspace;           // kAttnList: tile list + count
+  float scale;
+  int* status;
+  int num_sms;
+};
+
+size_t attn_list_workspace_bytes(int N, int G);
+// Builds tensor maps for q/k/v and launches.  Returns a cudaError_t value or
+// -1 if a tensor map could not be encoded.
+int launch_attention(const AttnLaunch& a, const void* q, const void* k, const void* v,
+                     cudaStream_t stream);
+
+// -------------------------------------------------------------- selector
+struct SelectLaunch {
+  int B, H, G, nK, n_exact, n_sample;
+  uint64_t seed;
+  const float* mass;
+  int32_t* idx;
+  float* log_w;
+  int* status;
+};
+int launch_select(const SelectLaunch& s, cudaStream_t stream);
+
+// ---------------------------------------------------------------- scorer
+struct ScoreLaunch {
+  int B, H, N, D, G, Bk, q_block, C, iters;
+  const int32_t* q_offsets;  // device or NULL
+  float scale;
+  const void* q;
+  const void* k;
+  float* mass;
+  float* centroids;   // [B,H,G,C,D]
+  int32_t* counts;    // [B,H,G,C]
+  float* kbar;        // [B,H,nK,D] scratch
+  float* stats;       // [B,H,G,C,2] scratch
+  int* status;
+  int num_sms;
+};
+size_t score_workspace_bytes(int B, int H, int N, int D, int G, int Bk, int C);
+int launch_score(const ScoreLaunch& s, cudaStream_t stream);
+
+}  // namespace isa_impl

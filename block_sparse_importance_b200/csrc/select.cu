@@ -1,0 +1,315 @@
+// Plan selection: exact set + SIP sample, one CTA per (batch, head, group).
+//
+// "AB-Attention: Accurate Block Attention for Accelerating Video Diffusion
+// Transformers", discussion of Sampling with Inclusion-Probability weighting:
+// the scores set inclusion probabilities, highly scored blocks may always
+// enter, the sampler returns a fixed number of distinct blocks, and a block
+// drawn with probability pi counts 1/pi times.  "InstaGen" abstract: the
+// top-scoring blocks form an exact set, the rest is represented by a sample
+// drawn in proportion to estimated attention.
+//
+// Everything that decides membership is integer arithmetic, so the plan is
+// reproducible bit for bit:
+//   * exact set: radix select (4 x 8-bit passes) on the fp32 bit patterns of
+//     the mass (monotone for non-negative values), ties to the lower block;
+//   * weights of the rest: w = floor(m / m_max * 2^31) + 1 in IEEE fp64;
+//   * capping at pi = 1: repeat { T = sum of uncapped w, n' = n_s - #capped,
+//     cap every block with n' w >= T } until stable (exact 64-bit sums);
+//   * systematic PPS over the uncapped blocks in ascending order with one
+//     uniform U = hi32(Philox4x64-10(key (seed,0), counter (g,h,b,0))[0]):
+//     with q = floor(x n' / T) and r = x n' mod T, the number of points
+//     (i + U 2^-32) T / n' below x is q + [r 2^32 > U T]; block j is drawn
+//     when that count steps between W_{j-1} and W_j;
+//   * drawn blocks get log_w = ln T - ln(n' w) (fp64, stored fp32).
+
+#include <cstdint>
+
+#include "isa_internal.h"
+
+namespace isa_impl {
+namespace {
+
+constexpr int kSelThreads = 256;
+constexpr int kSelWarps = kSelThreads / 32;
+
+// Philox4x64-10 (Salmon et al., SC'11), written for the device.
+__device__ __forceinline__ uint64_t philox_word0(uint64_t c0, uint64_t c1, uint64_t c2, uint64_t c3,
+                                                 uint64_t k0, uint64_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t lo0 = 0xD2E7470EE14C6C93ULL * c0, hi0 = __umul64hi(0xD2E7470EE14C6C93ULL, c0);
+    const uint64_t lo1 = 0xCA5A826395121157ULL * c2, hi1 = __umul64hi(0xCA5A826395121157ULL, c2);
+    const uint64_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+    k0 += 0x9E3779B97F4A7C15ULL;
+    k1 += 0xBB67AE8584CAA73BULL;
+  }
+  return c0;
+}
+
+struct SelShared {
+  uint64_t red64[kSelWarps];
+  uint32_t red32[kSelWarps];
+  uint32_t hist[256];
+  uint32_t sel_bin, remaining;
+  int bad;
+};
+
+__device__ __forceinline__ uint64_t block_sum_u64(uint64_t v, SelShared& sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) sh.red64[w] = v;
+  __syncthreads();
+  uint64_t t = 0;
+#pragma unroll
+  for (int i = 0; i < kSelWarps; ++i) t += sh.red64[i];
+  return t;
+}
+
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, SelShared& sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) sh.red32[w] = v;
+  __syncthreads();
+  uint32_t t = 0;
+#pragma unroll
+  for (int i = 0; i < kSelWarps; ++i) t = max(t, sh.red32[i]);
+  return t;
+}
+
+// Exclusive prefix sum over the block in thread order; returns the prefix of
+// this thread and writes the block total to *total.
+__device__ __forceinline__ uint64_t block_scan_u64(uint64_t v, SelShared& sh, uint64_t* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint64_t inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  __syncthreads();
+  if (lane == 31) sh.red64[w] = inc;
+  __syncthreads();
+  uint64_t before = 0, all = 0;
+#pragma unroll
+  for (int i = 0; i < kSelWarps; ++i) {
+    if (i < w) before += sh.red64[i];
+    all += sh.red64[i];
+  }
+  *total = all;
+  return before + inc - v;
+}
+
+// flags: bit0 exact, bit1 capped, bit2 drawn
+__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ SelShared sh;
+  const int nK = a.nK;
+  uint32_t* key = reinterpret_cast<uint32_t*>(sm);
+  uint32_t* wq = key + nK;
+  uint8_t* flag = reinterpret_cast<uint8_t*>(wq + nK);
+  const int tid = threadIdx.x;
+  const int64_t row = blockIdx.x;
+  const int g = static_cast<int>(row % a.G);
+  const int h = static_cast<int>((row / a.G) % a.H);
+  const int b = static_cast<int>(row / (static_cast<int64_t>(a.G) * a.H));
+  const float* m = a.mass + row * nK;
+  const int S = a.n_exact + a.n_sample;
+
+  if (tid == 0) sh.bad = 0;
+  __syncthreads();
+  for (int i = tid; i < nK; i += kSelThreads) {
+    const float v = m[i];
+    uint32_t k = 0;
+    if (!isfinite(v)) {
+      sh.bad = 1;
+    } else if (v > 0.0f) {
+      k = __float_as_uint(v);
+    }
+    key[i] = k;
+    flag[i] = 0;
+  }
+  __syncthreads();
+
+  // ---- exact set: the n_exact largest keys, ties to the lower index
+  if (a.n_exact > 0) {
+    uint32_t prefix = 0, mask = 0;
+    if (tid == 0) sh.remaining = a.n_exact;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kSelThreads) sh.hist[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < nK; i += kSelThreads)
+        if ((key[i] & mask) == prefix) atomicAdd(&sh.hist[(key[i] >> shift) & 255u], 1u);
+      __syncthreads();
+      if (tid < 32) {
+        // lane l owns bins [8l, 8l+8); suffix sums from the top bin down
+        uint32_t local = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) local += sh.hist[8 * tid + i];
+        uint32_t suf = local;  // sum of bins owned by lanes >= tid
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t t = __shfl_down_sync(0xffffffffu, suf, o);
+          if (tid + o < 32) suf += t;
+        }
+        const uint32_t need = sh.remaining;
+        const uint32_t above = suf - local;  // bins of higher lanes
+        const bool here = above < need && suf >= need;
+        if (here) {
+          uint32_t acc = above;
+          for (int i = 7; i >= 0; --i) {
+            const uint32_t c = sh.hist[8 * tid + i];
+            if (acc + c >= need) {
+              sh.sel_bin = 8 * tid + i;
+              sh.remaining = need - acc;
+              break;
+            }
+            acc += c;
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= sh.sel_bin << shift;
+      mask |= 255u << shift;
+      __syncthreads();
+    }
+    const uint32_t thr = prefix;
+    const uint32_t take_ties = sh.remaining;
+    uint64_t carry = 0;
+    for (int base = 0; base < nK; base += kSelThreads) {
+      const int i = base + tid;
+      const uint32_t k = i < nK ? key[i] : 0u;
+      const bool tie = i < nK && k == thr;
+      uint64_t tot;
+      const uint64_t rank = carry + block_scan_u64(tie ? 1u : 0u, sh, &tot);
+      if (i < nK && (k > thr || (tie && rank < take_ties))) flag[i] = 1;
+      carry += tot;
+    }
+    __syncthreads();
+  }
+
+  // ---- weights and capping over the rest
+  const int n_rest = nK - a.n_exact;
+  int n_left = 0;
+  uint64_t T = 0;
+  if (a.n_sample >= n_rest) {
+    for (int i = tid; i < nK; i += kSelThreads)
+      if (!(flag[i] & 1)) flag[i] |= 2;
+    __syncthreads();
+  } else if (a.n_sample > 0) {
+    uint32_t kmax = 0;
+    for (int i = tid; i < nK; i += kSelThreads)
+      if (!(flag[i] & 1)) kmax = max(kmax, key[i]);
+    kmax = block_max_u32(kmax, sh);
+    const double mmax = static_cast<double>(__uint_as_float(kmax));
+    for (int i = tid; i < nK; i += kSelThreads) {
+      uint32_t w = 0;
+      if (!(flag[i] & 1))
+        w = mmax > 0.0 ? static_cast<uint32_t>(floor(static_cast<double>(__uint_as_float(key[i])) / mmax *
+                                                     2147483648.0)) + 1u
+                       : 1u;
+      wq[i] = w;
+    }
+    __syncthreads();
+    int n_capped = 0;
+    for (;;) {
+      uint64_t t = 0;
+      for (int i = tid; i < nK; i += kSelThreads)
+        if (!(flag[i] & 3)) t += wq[i];
+      T = block_sum_u64(t, sh);
+      n_left = a.n_sample - n_capped;
+      uint64_t add = 0;
+      for (int i = tid; i < nK; i += kSelThreads)
+        if (!(flag[i] & 3) && static_cast<uint64_t>(n_left) * wq[i] >= T) ++add;
+      add = block_sum_u64(add, sh);  // all counts are taken before any flag changes
+      if (add == 0) break;
+      for (int i = tid; i < nK; i += kSelThreads)
+        if (!(flag[i] & 3) && static_cast<uint64_t>(n_left) * wq[i] >= T) flag[i] |= 2;
+      n_capped += static_cast<int>(add);
+      __syncthreads();
+    }
+    if (n_left > 0) {
+      const uint32_t U = static_cast<uint32_t>(
+          philox_word0(static_cast<uint32_t>(g), static_cast<uint32_t>(h), static_cast<uint32_t>(b), 0, a.seed, 0) >>
+          32);
+      const uint64_t nl = static_cast<uint64_t>(n_left);
+      const uint64_t ut_lo = static_cast<uint64_t>(U) * T;  // U T < 2^76
+      const uint64_t ut_hi = __umul64hi(static_cast<uint64_t>(U), T);
+      // points of the systematic comb below x
+      auto below = [&](uint64_t x) -> uint64_t {
+        const uint64_t xn = x * nl;  // < 2^57
+        const uint64_t q = xn / T, r = xn - q * T;
+        const uint64_t r_hi = r >> 32, r_lo = r << 32;  // r * 2^32
+        const bool gt = r_hi > ut_hi || (r_hi == ut_hi && r_lo > ut_lo);
+        return q + (gt ? 1u : 0u);
+      };
+      uint64_t carry = 0;
+      for (int base = 0; base < nK; base += kSelThreads) {
+        const int i = base + tid;
+        const bool unc = i < nK && !(flag[i] & 3);
+        const uint64_t w = unc ? wq[i] : 0u;
+        uint64_t tot;
+        const uint64_t W_prev = carry + block_scan_u64(w, sh, &tot);
+        if (unc && below(W_prev + w) != below(W_prev)) flag[i] |= 4;
+        carry += tot;
+      }
+      __syncthreads();
+    }
+  }
+
+  // ---- write the plan row: exact ascending, then capped + drawn ascending
+  int32_t* out_idx = a.idx + row * S;
+  float* out_lw = a.log_w + row * S;
+  const double lnT = T > 0 ? log(static_cast<double>(T)) : 0.0;
+  uint64_t c_exact = 0, c_rest = static_cast<uint64_t>(a.n_exact);
+  for (int base = 0; base < nK; base += kSelThreads) {
+    const int i = base + tid;
+    const uint8_t f = i < nK ? flag[i] : 0;
+    uint64_t tot_e, tot_r;
+    const uint64_t pe = block_scan_u64((f & 1) ? 1u : 0u, sh, &tot_e);
+    const uint64_t pr = block_scan_u64((f & 6) ? 1u : 0u, sh, &tot_r);
+    if (f & 1) {
+      const uint64_t o = c_exact + pe;
+      if (o < static_cast<uint64_t>(a.n_exact)) {
+        out_idx[o] = i;
+        out_lw[o] = 0.0f;
+      }
+    } else if (f & 6) {
+      const uint64_t o = c_rest + pr;
+      if (o < static_cast<uint64_t>(S)) {
+        out_idx[o] = i;
+        out_lw[o] = (f & 4) ? static_cast<float>(lnT - log(static_cast<double>(static_cast<uint64_t>(n_left) * wq[i])))
+                            : 0.0f;
+      }
+    }
+    c_exact += tot_e;
+    c_rest += tot_r;
+  }
+  if (tid == 0) {
+    if (sh.bad || c_exact != static_cast<uint64_t>(a.n_exact) || c_rest != static_cast<uint64_t>(S))
+      atomicCAS(a.status, 0, kStatusDeviceCheck);
+  }
+}
+
+}  // namespace
+
+int launch_select(const SelectLaunch& s, cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(s.nK) * 9 + 16;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  const long long rows = static_cast<long long>(s.B) * s.H * s.G;
+  select_kernel<<<static_cast<unsigned>(rows), kSelThreads, smem, stream>>>(s);
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace isa_impl

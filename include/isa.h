@@ -1,0 +1,233 @@
+/*
+ * isa.h -- C ABI of libisa.so: importance-sampled block-sparse attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (pages cited by title and section):
+ *   "AB-Attention: Accurate Block Attention for Accelerating Video Diffusion
+ *   Transformers" -- abstract, and the discussion of the Intra-Block Clustering
+ *   Selector (IBCS), Sampling with Inclusion-Probability weighting (SIP), the
+ *   logit-shift form of the weights, and fine-grained selection with tiled
+ *   execution;
+ *   "InstaGen: Group-Shared Importance Sampling for Fast Video Generation" --
+ *   abstract: block selection as importance sampling (exact set + a sample
+ *   reweighted by inverse probability), one sample shared per query cluster.
+ *
+ * Pipeline: isa_score (estimated attention mass per query group and key
+ * block) -> isa_select (plan: exact top blocks + a capped systematic PPS
+ * sample with log(1/pi) weights) -> isa_attention (one sparse flash-attention
+ * pass over the plan).  isa_dense_attention is the 100%-density limit.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, unless a
+ *     parameter says "host".  The library never allocates or frees memory in a
+ *     call; isa_create allocates the context's 4-byte device status word.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream) and returns after enqueueing.
+ *   - Host-side checks (shapes, null pointers, 16-byte alignment, budgets) are
+ *     made before anything is enqueued; a failing call returns
+ *     ISA_ERR_INVALID_ARG / ISA_ERR_UNSUPPORTED, enqueues nothing, and
+ *     isa_last_error() says why.
+ *   - Problems only the device can see (a block index out of range,
+ *     non-finite mass, malformed group offsets, a pipeline wait that ran out)
+ *     set the context's device status word; the kernel finishes without a
+ *     fault.  isa_sync_status() synchronises the stream and returns (and
+ *     clears) that word.
+ *   - Layouts are contiguous row-major:
+ *       Q, K, V, O   [B, H, N, d]  bf16
+ *       mass         [B, H, G, nK] fp32       nK = ceil(N / k_block)
+ *       idx, log_w   [B, H, G, S]  int32, fp32 S = n_exact + n_sample
+ *       lse          [B, H, N]     fp32 (natural log)
+ *   - A context serves one device; calls on one context are not thread-safe
+ *     with respect to each other's status word.
+ */
+#ifndef ISA_H_
+#define ISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ISA_API __attribute__((visibility("default")))
+#else
+#define ISA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum isa_status {
+  ISA_OK = 0,
+  ISA_ERR_INVALID_ARG = 1,  /* bad shape, pointer, alignment or budget      */
+  ISA_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. head_dim 96)        */
+  ISA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed             */
+  ISA_ERR_TIMEOUT = 4,      /* device: a pipeline wait ran out (no fault)    */
+  ISA_ERR_DEVICE_CHECK = 5  /* device: bad index / offsets / non-finite mass */
+} isa_status;
+
+typedef struct isa_context isa_context;
+
+/* Problem shape shared by all calls.
+ * Query groups: when q_offsets == NULL the groups are uniform blocks of
+ * q_block rows, group g = rows [g*q_block, min((g+1)*q_block, N)) and
+ * num_groups must equal ceil(N / q_block).  Otherwise group g is the cluster
+ * of rows [q_offsets[g], q_offsets[g+1]) of a permuted layout ("each query
+ * cluster draws one sample shared by all its queries", InstaGen abstract);
+ * q_offsets is a DEVICE int32 array of num_groups+1 entries with
+ * q_offsets[0] = 0, q_offsets[G] = N, strictly increasing (checked on the
+ * device).  The same groups apply to every batch entry and head.
+ * Key blocks: block b = rows [b*k_block, min((b+1)*k_block, N)); the last
+ * block may be partial.  Small key blocks are gathered into 128-row tiles by
+ * the attention kernel ("fine-grained selection with tiled execution"). */
+typedef struct isa_shape {
+  int32_t batch;             /* B >= 1                                   */
+  int32_t heads;             /* H >= 1                                   */
+  int32_t seq_len;           /* N >= 1                                   */
+  int32_t head_dim;          /* d: 64 or 128                             */
+  int32_t q_block;           /* uniform group rows, >= 1 (ignored if q_offsets) */
+  int32_t k_block;           /* 16, 32, 64 or 128                        */
+  int32_t num_groups;        /* G                                        */
+  const int32_t* q_offsets;  /* device [G+1] or NULL                     */
+  float scale;               /* logit scale, normally 1/sqrt(d)          */
+} isa_shape;
+
+/* Sampling parameters of the fused pipeline calls. */
+typedef struct isa_params {
+  int32_t n_clusters;  /* C: k-means clusters per query group, 1..16     */
+  int32_t n_iters;     /* I: k-means iterations, 1..16                   */
+  int32_t n_exact;     /* k_e: exact top blocks per group                */
+  int32_t n_sample;    /* n_s: sampled blocks per group                  */
+  uint64_t seed;       /* Philox key of the per-group uniforms           */
+} isa_params;
+
+/* Create a context on CUDA device `device` (allocates its 4-byte device
+ * status word).  *out receives the context.  Returns ISA_ERR_CUDA if the
+ * device cannot be used, ISA_ERR_UNSUPPORTED if it is not sm_100. */
+ISA_API isa_status isa_create(int device, isa_context** out);
+
+/* Destroy a context (frees its status word).  NULL is allowed. */
+ISA_API void isa_destroy(isa_context* ctx);
+
+/* Static string for a status code. */
+ISA_API const char* isa_status_string(isa_status status);
+
+/* Message of the last host-side failure on this context ("" if none). */
+ISA_API const char* isa_last_error(const isa_context* ctx);
+
+/* Synchronise `stream`, then return and clear the device status word
+ * (ISA_OK, ISA_ERR_TIMEOUT or ISA_ERR_DEVICE_CHECK), or ISA_ERR_CUDA if the
+ * stream reported an error. */
+ISA_API isa_status isa_sync_status(isa_context* ctx, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * isa_score -- IBCS block scorer ("AB-Attention", Intra-Block Clustering
+ * Selector: queries are clustered only within each query block; each cluster
+ * gets a representative and a weight equal to its size; the representatives
+ * score small key blocks without permuting tokens).
+ *   kbar_b   = mean of the valid rows of key block b, L_b = their count;
+ *   mu_c,n_c = Lloyd's k-means in each query group: init mu_c = row
+ *              floor(c*n_g/C) of the group, n_iters rounds of (assign to the
+ *              nearest centroid, ties to the lower c; move non-empty centroids
+ *              to the mean of their rows); n_c = sizes of the last assignment;
+ *   mass     = sum_c n_c * softmax_b(scale * mu_c . kbar_b + ln L_b),
+ *              so every mass row sums to the group's row count.
+ * q, k: [B,H,N,d] bf16.  mass: [B,H,G,nK] fp32 (written).
+ * centroids: optional [B,H,G,C,d] fp32 output, counts: optional [B,H,G,C]
+ * int32 output (NULL to skip).  workspace: device scratch of at least
+ * isa_score_workspace_bytes(shape, n_clusters) bytes, 256-byte aligned.
+ * 1 <= n_clusters <= 16, 1 <= n_iters <= 16.  A group with fewer rows than
+ * clusters is allowed (duplicate initial centroids stay empty).
+ * ------------------------------------------------------------------------- */
+ISA_API size_t isa_score_workspace_bytes(const isa_shape* shape, int32_t n_clusters);
+ISA_API isa_status isa_score(isa_context* ctx, const isa_shape* shape, const void* q, const void* k,
+                     int32_t n_clusters, int32_t n_iters, float* mass, float* centroids,
+                     int32_t* counts, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * isa_select -- exact set + SIP sample, one plan row per (batch, head, group)
+ * ("AB-Attention", Sampling with Inclusion-Probability weighting; "InstaGen"
+ * abstract).
+ *   exact set E = the n_exact largest mass values, ties to the lower block;
+ *   rest R: integer weights w_b = floor(m_b / max_R m * 2^31) + 1 (all 1 if
+ *   max_R m = 0), inclusion probabilities n' w_b / T capped at 1 by the
+ *   fixed-point iteration (capped blocks always enter, log_w = 0);
+ *   systematic PPS over the uncapped rest in ascending block order with one
+ *   Philox4x64-10 uniform per group (key (seed, 0), counter (g, h, b, 0),
+ *   U = high 32 bits of word 0), in exact 128-bit integer arithmetic;
+ *   drawn blocks carry log_w = ln T - ln(n' w_b) = ln(1/pi) (fp64, stored fp32).
+ *   Row layout: E ascending, then the capped and drawn blocks ascending.
+ *   If n_sample >= nK - n_exact every remaining block enters with log_w 0.
+ * mass: [B,H,G,nK] fp32 (non-finite values count as 0 and set
+ * ISA_ERR_DEVICE_CHECK).  idx: [B,H,G,S] int32, log_w: [B,H,G,S] fp32
+ * (written).  n_exact, n_sample >= 0, 1 <= n_exact + n_sample <= nK.
+ * The result is bit-identical to the CPU oracle for identical mass.
+ * ------------------------------------------------------------------------- */
+ISA_API isa_status isa_select(isa_context* ctx, const isa_shape* shape, const float* mass,
+                      int32_t n_exact, int32_t n_sample, uint64_t seed, int32_t* idx,
+                      float* log_w, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * isa_attention -- one sparse flash-attention pass over a plan
+ * ("AB-Attention": the weights become shifts of the sampled blocks' scores
+ * before the softmax, and only selected blocks receive exact attention; small
+ * key/value blocks are gathered into full tensor-core tiles).  For every
+ * query row r of group g:
+ *   z_k = scale * q_r . k_k + log_w[g][s]  for every valid row k of every
+ *         plan block idx[g][s], s < n_sel;
+ *   out_r = sum_k e^{z_k} v_k / sum_k e^{z_k};  lse_r = ln sum_k e^{z_k}.
+ * q, k, v: [B,H,N,d] bf16.  idx, log_w: [B,H,G,n_sel] (n_sel >= 1; a plan may
+ * be reused across calls).  out: [B,H,N,d] bf16 (written; every row of N is
+ * written exactly once).  lse: optional [B,H,N] fp32 (NULL to skip).
+ * workspace: device scratch of isa_attention_workspace_bytes(shape) bytes
+ * (0 when q_offsets == NULL; then workspace may be NULL).
+ * An idx entry outside [0, nK) is replaced by an empty block and sets
+ * ISA_ERR_DEVICE_CHECK.  All device pointers must be 16-byte aligned.
+ * ------------------------------------------------------------------------- */
+ISA_API size_t isa_attention_workspace_bytes(const isa_shape* shape);
+ISA_API isa_status isa_attention(isa_context* ctx, const isa_shape* shape, const void* q, const void* k,
+                         const void* v, const int32_t* idx, const float* log_w, int32_t n_sel,
+                         void* out, float* lse, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* ---------------------------------------------------------------------------
+ * isa_dense_attention -- the 100%-density limit: softmax(scale Q K^T) V over
+ * all keys, by the same tensor-core kernel with the whole sequence as plan
+ * and zero log-weights.  Groups are ignored.  q, k, v, out as in
+ * isa_attention; lse optional.
+ * ------------------------------------------------------------------------- */
+ISA_API isa_status isa_dense_attention(isa_context* ctx, const isa_shape* shape, const void* q,
+                               const void* k, const void* v, void* out, float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * isa_pipeline -- score -> select -> attention in one call on device
+ * buffers (the whole hot path of one attention layer).  The mass tensor,
+ * the plan and the scorer's scratch are carved from `workspace`
+ * (isa_pipeline_workspace_bytes bytes).  plan_idx / plan_log_w: optional
+ * device outputs [B,H,G,S] receiving the plan (NULL: kept in the workspace).
+ * ------------------------------------------------------------------------- */
+ISA_API size_t isa_pipeline_workspace_bytes(const isa_shape* shape, const isa_params* params);
+ISA_API isa_status isa_pipeline(isa_context* ctx, const isa_shape* shape, const isa_params* params,
+                        const void* q, const void* k, const void* v, void* out, float* lse,
+                        int32_t* plan_idx, float* plan_log_w, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * isa_pipeline_host -- the same from HOST buffers: copies q, k, v (host,
+ * [B,H,N,d] bf16; page-locked memory makes the copies asynchronous) into the
+ * device arena, runs the pipeline, and copies the output back to out_host
+ * ([B,H,N,d] bf16).  The arena holds Q, K, V, O and the pipeline workspace:
+ * isa_pipeline_host_workspace_bytes bytes.  shape->q_offsets stays a device
+ * pointer.  Enqueues everything on `stream`; out_host is valid after the
+ * stream is synchronised.
+ * ------------------------------------------------------------------------- */
+ISA_API size_t isa_pipeline_host_workspace_bytes(const isa_shape* shape, const isa_params* params);
+ISA_API isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, const isa_params* params,
+                             const void* q_host, const void* k_host, const void* v_host,
+                             void* out_host, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISA_H_ */

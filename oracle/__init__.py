@@ -22,9 +22,11 @@ _LIB = os.path.join(_HERE, "_isa_ref.so")
 _lock = threading.Lock()
 _lib = None
 
-# Margin below which a k-means assignment counts as a near tie (relative to
-# ||q||^2 + ||mu||^2): well above the rounding of a 128-term fp32 distance.
-KMEANS_TIE_REL = 1e-4
+# Margin below which a k-means assignment counts as a near tie, relative to
+# ||q||^2 + ||mu||^2.  A d-term fp32 sum of squares is within d 2^-24 of its
+# magnitude (<= 2 (||q||^2 + ||mu||^2)), i.e. 1.5e-5 of that scale at d = 128;
+# the threshold keeps a 2x margin over that bound.
+KMEANS_TIE_REL = 3e-5
 
 
 def build(force: bool = False) -> str:

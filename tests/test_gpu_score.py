@@ -1,0 +1,62 @@
+"""GPU parity of isa_score against the oracle: key means and k-means outputs
+per group (groups whose fp64 clustering met a near tie are checked for
+validity only), estimated mass within relative L2 1e-3."""
+import numpy as np
+import pytest
+import torch
+
+from tests import cases
+from tests.cases import Case
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def isa():
+    from block_sparse_importance_b200 import build, isa as m
+    build.build()
+    return m
+
+
+def _run(isa, c: Case):
+    q, k, _ = c.cuda()
+    lay = c.layout()
+    C = c.w.n_clusters
+    cen = torch.empty(1, c.H, c.G, C, c.d, device="cuda")
+    cnt = torch.empty(1, c.H, c.G, C, dtype=torch.int32, device="cuda")
+    mass = isa.score(q, k, lay, C, c.w.n_iters, centroids=cen, counts=cnt)
+    assert isa.context().sync_status() == isa.ISA_OK
+    m_ref, cen_ref, cnt_ref, amb = c.oracle_mass()
+    mass = mass.cpu().numpy().astype(np.float64)
+    cen = cen.cpu().numpy().astype(np.float64)
+    cnt = cnt.cpu().numpy()
+    sizes = np.diff(c.offsets)
+    assert np.all(cnt.sum(-1) == sizes[None, None, :])                 # valid everywhere
+    assert np.allclose(mass.sum(-1), sizes[None, None, :], rtol=1e-4)  # sum_b m = n_g
+    ok = ~amb
+    assert ok.mean() > 0.5
+    assert np.array_equal(cnt[ok], cnt_ref[ok])
+    live = (cnt_ref > 0)[..., None] & ok[..., None, None]
+    diff = np.abs(cen - cen_ref)
+    assert np.max(np.where(live, diff, 0)) < 1e-4 * max(1.0, np.abs(cen_ref).max())
+    r = cases.rel_l2(mass[ok], m_ref[ok])
+    assert r <= cases.MASS_REL_L2, r
+    return r
+
+
+@pytest.mark.parametrize("preset,N,Bk,Bq,C", [
+    ("tiny", 4096, 64, 64, 4),       # the tiny layer in full
+    ("wan13", 1500, 64, 128, 8),
+    ("wan13", 1200, 16, 128, 8),
+    ("wan13", 1000, 64, 100, 3),     # non-power-of-two clusters, ragged groups
+    ("wan13", 1000, 32, 128, 16),
+])
+def test_score_matches_oracle(isa, preset, N, Bk, Bq, C):
+    c = Case(preset, 2 if preset != "tiny" else 1, N, Bk, Bq, 2, 2, n_clusters=C)
+    _run(isa, c)
+
+
+def test_score_variable_clusters(isa):
+    off = cases.random_offsets(2000, 16, 600, seed=5)
+    c = Case("wan13", 2, 2000, 64, 128, 2, 2, offsets=off)
+    _run(isa, c)
