@@ -193,6 +193,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="wan14_10")
+    ap.add_argument("--heads", type=int, default=0, help="run only the first H heads (profiling cases)")
     ap.add_argument("--impl", default="isa", choices=["isa", "reference"])
     ap.add_argument("--ref-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -219,6 +220,8 @@ def main():
     torch.cuda.set_device(dev)
 
     w = wl.preset(args.workload, seed=0)
+    if args.heads:
+        w = wl.preset(args.workload, seed=0, heads=args.heads)
     inp = wl.make_inputs(w, str(dev))
     q, k, v = inp.q, inp.k, inp.v
     off_dev = torch.from_numpy(inp.offsets).to(dev) if w.variable_groups else None
