@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "isa.h"
 #include "isa_internal.h"
@@ -420,3 +421,71 @@ isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, const isa
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// isa_attention_noalloc: isa_attention for callers that cannot allocate.
+//
+// Some callers cannot hand this library any device memory of their own: a
+// framework custom-op or plugin interface that passes a kernel only its
+// inputs and outputs, or latency-critical code that must not call cudaMalloc
+// (which may synchronise the device) and has no workspace to lend.  For
+// them the tile-list scratch of the attention kernel (needed for variable
+// query clusters and for uniform groups of more than 128 rows) lives in the
+// file-scope array below instead of a caller workspace.
+//
+// The array is a module global: every GPU that loads this library holds its
+// kNoAllocScratchBytes until the process exits.  In host code its name is only
+// a host-side stand-in, so the device address is looked up with
+// cudaGetSymbolAddress the first time the entry point runs on a device (with
+// that device current) and cached per device.  Make that first call on each
+// device before any stream capture.  Every call shares the one array and it
+// keeps the last call's contents; the tile-list kernel rewrites every entry it
+// uses (and the count) on each call, so nothing needs clearing.  Calls whose
+// kernels overlap on the GPU (different streams, no ordering between them)
+// race on the array.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[64] = {nullptr};
+
+// Device address of the scratch array on `device` (which must be current).
+cudaError_t noalloc_scratch(int device, void** out) {
+  if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[device]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[device] = p;
+  }
+  *out = g_noalloc_ptr[device];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" isa_status isa_attention_noalloc(isa_context* ctx, const isa_shape* shape, const void* q, const void* k,
+                                            const void* v, const int32_t* idx, const float* log_w, int32_t n_sel,
+                                            void* out, float* lse, void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  const size_t need = attn_ws_bytes(shape);
+  if (need > kNoAllocScratchBytes)
+    return fail(ctx, ISA_ERR_INVALID_ARG,
+                "isa_attention_noalloc: the tile list needs %zu bytes, more than its built-in %zu-byte scratch "
+                "(num_groups + seq_len/128 must stay below %zu); use isa_attention with a workspace",
+                need, kNoAllocScratchBytes, kNoAllocScratchBytes / 16 - 1);
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  void* scratch = nullptr;
+  if (need) {
+    const cudaError_t e = noalloc_scratch(ctx->device, &scratch);
+    if (e != cudaSuccess)
+      return fail(ctx, ISA_ERR_CUDA, "isa_attention_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+  }
+  return do_attention(ctx, shape, q, k, v, idx, log_w, n_sel, out, lse, scratch, need ? kNoAllocScratchBytes : 0,
+                      false, static_cast<cudaStream_t>(stream));
+}

@@ -76,8 +76,9 @@ def lib():
             L.isa_pipeline_host_workspace_bytes.argtypes = [S, Pp]
             L.isa_pipeline_host_workspace_bytes.restype = _sz
             L.isa_pipeline_host.argtypes = [_P, S, Pp, _P, _P, _P, _P, _P, _sz, _P]
+            L.isa_attention_noalloc.argtypes = [_P, S, _P, _P, _P, _P, _P, _i32, _P, _P, _P]
             for name in ("isa_create", "isa_sync_status", "isa_score", "isa_select", "isa_attention",
-                         "isa_dense_attention", "isa_pipeline", "isa_pipeline_host"):
+                         "isa_dense_attention", "isa_pipeline", "isa_pipeline_host", "isa_attention_noalloc"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -310,3 +311,24 @@ def pipeline_host(q_host, k_host, v_host, out_host, lay: Layout, p: Params, work
                                  _ptr(v_host), _ptr(out_host), _ptr(workspace), nb, _stream(stream))
     ctx.check(st, "isa_pipeline_host")
     return out_host
+
+
+def attention_noalloc(q, k, v, idx, log_w, lay: Layout, out=None, lse=None, ctx: Optional[Context] = None,
+                      stream=None, want_lse: bool = False):
+    """isa_attention_noalloc: the same pass as attention(), for callers that
+    cannot allocate device memory (no workspace argument: the library's own
+    1 MiB scratch array holds the tile list).  Calls that overlap on the GPU
+    share that array, so keep them ordered."""
+    ctx = ctx or context(q.device.index or 0)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, torch.bfloat16, n)
+    _dev(idx, torch.int32, "idx")
+    _dev(log_w, torch.float32, "log_w")
+    out = out if out is not None else torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = _empty(q.shape[:3], torch.float32, q.device)
+    sh = lay.c()
+    st = lib().isa_attention_noalloc(ctx.handle, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
+                                     _ptr(log_w), int(idx.shape[-1]), _ptr(out), _ptr(lse), _stream(stream))
+    ctx.check(st, "isa_attention_noalloc")
+    return (out, lse) if want_lse else out

@@ -226,6 +226,28 @@ ISA_API isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, c
                              void* out_host, void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/* ---------------------------------------------------------------------------
+ * isa_attention_noalloc -- isa_attention for callers that cannot allocate.
+ * No counterpart in the pages: it is an interface convenience of this library.
+ * Some callers cannot give the library device memory: a framework custom-op
+ * or plugin interface that hands a kernel only its inputs and outputs, or
+ * latency-critical code that must not call cudaMalloc (which may synchronise
+ * the device).  This call computes exactly what isa_attention computes, with
+ * the same arguments minus the workspace; the tile list that variable
+ * clusters and groups of more than 128 rows need lives in a 1 MiB array
+ * inside the library, so num_groups + seq_len / 128 must stay below 65535
+ * (larger shapes return ISA_ERR_INVALID_ARG).  Every GPU that loads the
+ * library holds that 1 MiB until the process exits.  The first call on each
+ * device looks up the array's device address (make that first call before
+ * any stream capture).  All calls share the one array: calls whose kernels
+ * overlap on the GPU race on it, so order them (one stream, or events).  The
+ * call allocates nothing.
+ * ------------------------------------------------------------------------- */
+ISA_API isa_status isa_attention_noalloc(isa_context* ctx, const isa_shape* shape, const void* q,
+                                         const void* k, const void* v, const int32_t* idx,
+                                         const float* log_w, int32_t n_sel, void* out, float* lse,
+                                         void* stream);
+
 #ifdef __cplusplus
 }
 #endif
