@@ -66,6 +66,8 @@ struct AttnArgs {
   const int* tile_count;  // list mode
   float scale_log2;
   int* status;
+  uint64_t timeout;  // per-wait limit, ns
+  int stall;         // test hook (failure detection)
 };
 
 template <int D>
@@ -78,7 +80,8 @@ struct Layout {
   static constexpr uint32_t kBarOff = kRingOff + kRing * kKVBytes;
   static constexpr int kBarQFull = 0, kBarQEmpty = 2, kBarKVFull = 4, kBarKVEmpty = 4 + kRing,
                        kBarSFull = 4 + 2 * kRing, kBarPFull = kBarSFull + 2,
-                       kBarODone = kBarPFull + 2, kBarFinal = kBarODone + 2, kNumBars = kBarFinal + 1;
+                       kBarODone = kBarPFull + 2, kBarFinal = kBarODone + 2, kBarStall = kBarFinal + 1,
+                       kNumBars = kBarStall + 1;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kTotal = kMiscOff + 16;
   static constexpr uint32_t kAlloc = kTotal + 1024;
@@ -175,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(L::kBarKVEmpty + i), 1);
     }
     mbar_init(bar(L::kBarFinal), 1);
+    mbar_init(bar(L::kBarStall), 1);  // never arrived at: only the failure-detection hook waits on it
     *abort_flag = 0;
     *bad_index = 0;
     fence_mbar_init();
@@ -214,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!present) continue;
         uint32_t& q_loads = x ? q_loads1 : q_loads0;
         const Work& wx = x ? wk[1] : wk[0];
-        if (lane == 0) ok = mbar_wait(bar(L::kBarQEmpty + x), (q_loads & 1u) ^ 1u, abort_flag, kWaitTimeoutNs);
+        if (lane == 0) ok = mbar_wait(bar(L::kBarQEmpty + x), (q_loads & 1u) ^ 1u, abort_flag, a.timeout);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         ++q_loads;
@@ -231,9 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (shared && side == 1) return true;
         const Work& w = side ? wk[1] : wk[0];
         const uint32_t slot = ring_pos % kRing, use = ring_pos / kRing;
-        ++ring_pos;
         bool good = true;
-        if (lane == 0) good = mbar_wait(bar(L::kBarKVEmpty + slot), (use & 1u) ^ 1u, abort_flag, kWaitTimeoutNs);
+        if (lane == 0) good = mbar_wait(bar(L::kBarKVEmpty + slot), (use & 1u) ^ 1u, abort_flag, a.timeout);
         good = __shfl_sync(0xffffffffu, good, 0);
         if (!good) return false;
         if (lane == 0) mbar_arrive_expect_tx(bar(L::kBarKVFull + slot), L::kKVBytes);
@@ -262,10 +265,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(dst + c * L::kChunkBytes + lane * a.Bk * 128, map, bar(L::kBarKVFull + slot), c * 64, y,
                         w.bh);
         }
+        ++ring_pos;  // counts only items whose copies were issued
         return true;
       });
     }
-    if (!ok && lane == 0) {
+    if ((!ok || *abort_flag) && lane == 0) {
       // drain the copies still in flight before the CTA may exit
       const uint32_t first = ring_pos > kRing ? ring_pos - kRing : 0;
       for (uint32_t i = first; i < ring_pos; ++i) drain_wait(bar(L::kBarKVFull + i % kRing), (i / kRing) & 1u);
@@ -280,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ring_pos = 0, q_waits0 = 0, q_waits1 = 0, p_waits0 = 0, p_waits1 = 0;
       uint32_t last_k = 0, last_v = 0;
       bool ok = true;
+      if (a.stall) ok = mbar_wait(bar(L::kBarStall), 0, abort_flag, a.timeout);
       for (int p = blockIdx.x; p < n_pairs && ok; p += gridDim.x) {
         Work wk[2];
         const bool pr0 = decode_work(a, tph, n_work, 2 * p, wk[0]);
@@ -290,19 +295,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool release = !shared || side == 1;
           if (kind == 0 && j == 0) {
             uint32_t& qw = side ? q_waits1 : q_waits0;
-            if (!mbar_wait(bar(L::kBarQFull + side), qw & 1u, abort_flag, kWaitTimeoutNs)) return false;
+            if (!mbar_wait(bar(L::kBarQFull + side), qw & 1u, abort_flag, a.timeout)) return false;
             ++qw;
           }
           if (kind == 1) {
             uint32_t& pw = side ? p_waits1 : p_waits0;
-            if (!mbar_wait(bar(L::kBarPFull + side), pw & 1u, abort_flag, kWaitTimeoutNs)) return false;
+            if (!mbar_wait(bar(L::kBarPFull + side), pw & 1u, abort_flag, a.timeout)) return false;
             ++pw;
           }
           uint32_t slot;
           uint32_t& last = kind ? last_v : last_k;
           if (acquire) {
             slot = ring_pos % kRing;
-            if (!mbar_wait(bar(L::kBarKVFull + slot), (ring_pos / kRing) & 1u, abort_flag, kWaitTimeoutNs))
+            if (!mbar_wait(bar(L::kBarKVFull + slot), (ring_pos / kRing) & 1u, abort_flag, a.timeout))
               return false;
             ++ring_pos;
             last = slot;
@@ -376,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (!mbar_wait(bar(L::kBarSFull + x), s_waits & 1u, abort_flag, kWaitTimeoutNs)) {
+        if (!mbar_wait(bar(L::kBarSFull + x), s_waits & 1u, abort_flag, a.timeout)) {
           ok = false;
           break;
         }
@@ -454,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(L::kBarPFull + x));
       }
       if (!ok) break;
-      if (!mbar_wait(bar(L::kBarODone + x), o_waits & 1u, abort_flag, kWaitTimeoutNs)) {
+      if (!mbar_wait(bar(L::kBarODone + x), o_waits & 1u, abort_flag, a.timeout)) {
         ok = false;
         break;
       }
@@ -590,6 +595,8 @@ int launch_d(const AttnLaunch& l, const void* q, const void* k, const void* v, c
   a.lse = l.lse;
   a.scale_log2 = l.scale * kLog2e;
   a.status = l.status;
+  a.timeout = l.wait_timeout_ns ? l.wait_timeout_ns : kWaitTimeoutNs;
+  a.stall = l.stall;
   int tiles_upper;
   if (l.mode == kAttnDense) {
     a.tiles_per_head = (l.N + kTileRows - 1) / kTileRows;

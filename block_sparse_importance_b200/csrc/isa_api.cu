@@ -18,6 +18,8 @@ struct isa_context {
   int device;
   int num_sms;
   int* d_status;
+  uint64_t wait_timeout_ns;  // 0: the kernels' default
+  int stall_attention;       // failure-detection test hook
   char last_error[512];
 };
 
@@ -196,6 +198,8 @@ isa_status do_attention(isa_context* ctx, const isa_shape* s, const void* q, con
   l.scale = s->scale;
   l.status = ctx->d_status;
   l.num_sms = ctx->num_sms;
+  l.wait_timeout_ns = ctx->wait_timeout_ns;
+  l.stall = ctx->stall_attention;
   if (dense) {
     l.mode = kAttnDense;
     l.S = 1;
@@ -282,6 +286,8 @@ isa_status isa_create(int device, isa_context** out) {
     c->device = device;
     c->num_sms = prop.multiProcessorCount;
     c->d_status = d_status;
+    c->wait_timeout_ns = 0;
+    c->stall_attention = 0;
     c->last_error[0] = 0;
     *out = c;
   } else if (d_status) {
@@ -326,6 +332,15 @@ isa_status isa_sync_status(isa_context* ctx, void* stream) {
   if (h == ISA_ERR_TIMEOUT) return ISA_ERR_TIMEOUT;
   if (h != 0) return ISA_ERR_DEVICE_CHECK;
   return ISA_OK;
+}
+
+isa_status isa_debug_set(isa_context* ctx, int32_t knob, uint64_t value) {
+  if (!ctx) return ISA_ERR_INVALID_ARG;
+  switch (knob) {
+    case ISA_DEBUG_WAIT_TIMEOUT_NS: ctx->wait_timeout_ns = value; return ISA_OK;
+    case ISA_DEBUG_STALL_ATTENTION: ctx->stall_attention = value != 0; return ISA_OK;
+  }
+  return fail(ctx, ISA_ERR_INVALID_ARG, "isa_debug_set: unknown knob %d", knob);
 }
 
 size_t isa_score_workspace_bytes(const isa_shape* s, int32_t n_clusters) {

@@ -34,6 +34,8 @@ struct AttnLaunch {
   float scale;
   int* status;
   int num_sms;
+  uint64_t wait_timeout_ns;  // per-wait limit of the bounded pipeline waits
+  int stall;                 // test hook: the MMA warp waits on a barrier nothing arrives at
 };
 
 size_t attn_list_workspace_bytes(int N, int G);

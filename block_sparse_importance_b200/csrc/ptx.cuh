@@ -47,15 +47,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase with parity `parity` of barrier `bar` has completed.
 // Every wait is bounded: it gives up when *abort becomes non-zero (another
-// role of the CTA gave up) or when `deadline_ns` of the global timer passes,
-// in which case it sets *abort itself.  Returns false if it gave up.
+// role of the CTA gave up) or when more than `timeout_ns` of the global timer
+// have passed since the wait began, in which case it sets *abort itself.
+// Returns false if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          uint64_t deadline_ns) {
+                                          uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if ((++spins & 63u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() > deadline_ns) {
+      if (global_timer_ns() - t0 > timeout_ns) {
         *abort = 1;
         return false;
       }

@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libisa.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "isa.h")
 
 ISA_OK, ISA_ERR_INVALID_ARG, ISA_ERR_UNSUPPORTED, ISA_ERR_CUDA, ISA_ERR_TIMEOUT, ISA_ERR_DEVICE_CHECK = range(6)
+ISA_DEBUG_WAIT_TIMEOUT_NS, ISA_DEBUG_STALL_ATTENTION = 1, 2
 
 _i32, _u64, _f32, _P, _sz = ctypes.c_int32, ctypes.c_uint64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -76,6 +77,8 @@ def lib():
             L.isa_pipeline_host_workspace_bytes.argtypes = [S, Pp]
             L.isa_pipeline_host_workspace_bytes.restype = _sz
             L.isa_pipeline_host.argtypes = [_P, S, Pp, _P, _P, _P, _P, _P, _sz, _P]
+            L.isa_debug_set.argtypes = [_P, _i32, _u64]
+            L.isa_debug_set.restype = ctypes.c_int
             L.isa_attention_noalloc.argtypes = [_P, S, _P, _P, _P, _P, _P, _i32, _P, _P, _P]
             for name in ("isa_create", "isa_sync_status", "isa_score", "isa_select", "isa_attention",
                          "isa_dense_attention", "isa_pipeline", "isa_pipeline_host", "isa_attention_noalloc"):
@@ -120,6 +123,10 @@ class Context:
         if status != ISA_OK:
             msg = lib().isa_last_error(self.handle).decode()
             raise IsaError(status, "%s: %s: %s" % (what, status_string(status), msg))
+
+    def debug_set(self, knob: int, value: int):
+        """Failure-detection test hooks (ISA_DEBUG_* in include/isa.h)."""
+        self.check(lib().isa_debug_set(self.handle, knob, value), "isa_debug_set")
 
     def sync_status(self, stream: Optional[torch.cuda.Stream] = None) -> int:
         """Synchronise the stream; return (and clear) the device status word."""

@@ -227,6 +227,21 @@ ISA_API isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, c
                              void* stream);
 
 /* ---------------------------------------------------------------------------
+ * isa_debug_set -- test hooks for failure detection (not for production use).
+ *   ISA_DEBUG_WAIT_TIMEOUT_NS: per-wait time limit, in ns, of every bounded
+ *     pipeline wait in kernels launched on this context (default 2e9; 0
+ *     restores the default).
+ *   ISA_DEBUG_STALL_ATTENTION: when non-zero, attention launches on this
+ *     context make their MMA warp wait on a barrier that nothing arrives at;
+ *     the wait runs out after the per-wait limit, every CTA takes its abort
+ *     path (drains in-flight copies, frees tensor memory) and the status word
+ *     reads ISA_ERR_TIMEOUT.  The outputs of such a launch are undefined.
+ * Returns ISA_ERR_INVALID_ARG for an unknown knob.
+ * ------------------------------------------------------------------------- */
+enum { ISA_DEBUG_WAIT_TIMEOUT_NS = 1, ISA_DEBUG_STALL_ATTENTION = 2 };
+ISA_API isa_status isa_debug_set(isa_context* ctx, int32_t knob, uint64_t value);
+
+/* ---------------------------------------------------------------------------
  * isa_attention_noalloc -- isa_attention for callers that cannot allocate.
  * No counterpart in the pages: it is an interface convenience of this library.
  * Some callers cannot give the library device memory: a framework custom-op
