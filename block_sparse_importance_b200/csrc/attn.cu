@@ -391,20 +391,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         // sequence (a partial tail block) needs per-element masking
         if (c_valid == 0) c_bias = -INFINITY;
         const bool partial = __any_sync(0xffffffffu, c_valid > 0 && c_valid < 16);
-        // pass 1: row max of z = scale*s + log_w (log2 units) over valid keys
+        // pass 1: row max of z = scale*s + log_w (log2 units) over valid keys.
+        // scale > 0, so the max of z over a 16-column chunk is scale * (max of
+        // s) + bias; eight independent accumulators keep the chain short, and
+        // the next chunk's TMEM load is in flight while this one is reduced.
         float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32];
-          tmem_ld32(lane_base + col_s + 32 * c, sv);
-          const float b0 = __shfl_sync(0xffffffffu, c_bias, 2 * c), b1 = __shfl_sync(0xffffffffu, c_bias, 2 * c + 1);
-          const int n0 = __shfl_sync(0xffffffffu, c_valid, 2 * c), n1 = __shfl_sync(0xffffffffu, c_valid, 2 * c + 1);
+        {
+          uint32_t sv[2][32];
+          tmem_ld32(lane_base + col_s, sv[0]);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float z = fmaf(__uint_as_float(sv[i]), a.scale_log2, i < 16 ? b0 : b1);
-            if (partial) z = (i & 15) < (i < 16 ? n0 : n1) ? z : -INFINITY;
-            mx = fmaxf(mx, z);
+          for (int c = 0; c < 4; ++c) {
+            if (c < 3) tmem_ld32(lane_base + col_s + 32 * (c + 1), sv[(c + 1) & 1]);
+            const uint32_t* v = sv[c & 1];
+            const float b0 = __shfl_sync(0xffffffffu, c_bias, 2 * c);
+            const float b1 = __shfl_sync(0xffffffffu, c_bias, 2 * c + 1);
+            float h[2];
+            if (!partial) {
+              float l4[4], h4[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                l4[i] = fmaxf(fmaxf(__uint_as_float(v[i]), __uint_as_float(v[i + 4])),
+                              fmaxf(__uint_as_float(v[i + 8]), __uint_as_float(v[i + 12])));
+                h4[i] = fmaxf(fmaxf(__uint_as_float(v[16 + i]), __uint_as_float(v[20 + i])),
+                              fmaxf(__uint_as_float(v[24 + i]), __uint_as_float(v[28 + i])));
+              }
+              h[0] = fmaxf(fmaxf(l4[0], l4[1]), fmaxf(l4[2], l4[3]));
+              h[1] = fmaxf(fmaxf(h4[0], h4[1]), fmaxf(h4[2], h4[3]));
+            } else {
+              const int n0 = __shfl_sync(0xffffffffu, c_valid, 2 * c), n1 = __shfl_sync(0xffffffffu, c_valid, 2 * c + 1);
+              h[0] = -INFINITY;
+              h[1] = -INFINITY;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const bool ok_i = (i & 15) < (i < 16 ? n0 : n1);
+                if (ok_i) h[i >> 4] = fmaxf(h[i >> 4], __uint_as_float(v[i]));
+              }
+            }
+            mx = fmaxf(mx, fmaxf(fmaf(h[0], a.scale_log2, b0), fmaf(h[1], a.scale_log2, b1)));
+            if (c < 3) tmem_wait_ld();
           }
         }
         if (j == 0) {
@@ -427,32 +452,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
         // pass 2: P = exp2(z - max) as bf16 pairs; chunk c's 16 packed
-        // columns land on columns 16c.. of S, which earlier chunks already read
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32];
-          tmem_ld32(lane_base + col_s + 32 * c, sv);
-          const float bm0 = __shfl_sync(0xffffffffu, c_bias, 2 * c) - m_used;
-          const float bm1 = __shfl_sync(0xffffffffu, c_bias, 2 * c + 1) - m_used;
-          const int n0 = __shfl_sync(0xffffffffu, c_valid, 2 * c), n1 = __shfl_sync(0xffffffffu, c_valid, 2 * c + 1);
-          tmem_wait_ld();
-          uint32_t pk[16];
+        // columns land on columns 16c.. of S, which earlier chunks already
+        // read.  The next chunk's load overlaps this chunk's exponentials.
+        {
+          float ls[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e0 = 2 * i, e1 = e0 + 1;  // column within this 32-column chunk
-            const float bm = i < 8 ? bm0 : bm1;
-            const int nv = i < 8 ? n0 : n1;
-            float x0 = fmaf(__uint_as_float(sv[2 * i]), a.scale_log2, bm);
-            float x1 = fmaf(__uint_as_float(sv[2 * i + 1]), a.scale_log2, bm);
-            if (partial) {
-              x0 = (e0 & 15) < nv ? x0 : -INFINITY;
-              x1 = (e1 & 15) < nv ? x1 : -INFINITY;
+          for (int i = 0; i < 8; ++i) ls[i] = 0.0f;
+          uint32_t sv[2][32];
+          tmem_ld32(lane_base + col_s, sv[0]);
+          tmem_wait_ld();
+#pragma unroll 2
+          for (int c = 0; c < 4; ++c) {
+            if (c < 3) tmem_ld32(lane_base + col_s + 32 * (c + 1), sv[(c + 1) & 1]);
+            const uint32_t* v = sv[c & 1];
+            const float bm0 = __shfl_sync(0xffffffffu, c_bias, 2 * c) - m_used;
+            const float bm1 = __shfl_sync(0xffffffffu, c_bias, 2 * c + 1) - m_used;
+            const int n0 = __shfl_sync(0xffffffffu, c_valid, 2 * c), n1 = __shfl_sync(0xffffffffu, c_valid, 2 * c + 1);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int e0 = 2 * i, e1 = e0 + 1;  // column within this 32-column chunk
+              const float bm = i < 8 ? bm0 : bm1;
+              const int nv = i < 8 ? n0 : n1;
+              float x0 = fmaf(__uint_as_float(v[e0]), a.scale_log2, bm);
+              float x1 = fmaf(__uint_as_float(v[e1]), a.scale_log2, bm);
+              if (partial) {
+                x0 = (e0 & 15) < nv ? x0 : -INFINITY;
+                x1 = (e1 & 15) < nv ? x1 : -INFINITY;
+              }
+              const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+              ls[i & 7] += p0 + p1;
+              pk[i] = pack_bf16x2(p0, p1);
             }
-            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-            l_sum += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+            tmem_st16(lane_base + col_s + 16 * c, pk);
+            if (c < 3) tmem_wait_ld();
           }
-          tmem_st16(lane_base + col_s + 16 * c, pk);
+          l_sum += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         }
         tmem_wait_st();
         tc_fence_before();

@@ -81,7 +81,8 @@ isa_status check_shape(isa_context* ctx, const isa_shape* s) {
     if (!aligned(s->q_offsets, 4)) return fail(ctx, ISA_ERR_INVALID_ARG, "q_offsets not 4-byte aligned");
     if (s->num_groups > s->seq_len) return fail(ctx, ISA_ERR_INVALID_ARG, "more groups than rows");
   }
-  if (!std::isfinite(s->scale)) return fail(ctx, ISA_ERR_INVALID_ARG, "scale must be finite");
+  if (!std::isfinite(s->scale) || !(s->scale > 0.0f))
+    return fail(ctx, ISA_ERR_INVALID_ARG, "scale must be finite and > 0");
   const long long bh = static_cast<long long>(s->batch) * s->heads;
   if (bh * s->seq_len > (1LL << 40) || bh > (1LL << 30))
     return fail(ctx, ISA_ERR_INVALID_ARG, "tensor too large");

@@ -1,0 +1,52 @@
+// Warp-level tensor-core helpers (mma.sync m16n8k16, bf16 in, fp32 out) and
+// ldmatrix loads, for the scorer's small per-group products.  Fragment
+// layouts follow the PTX ISA's description of mma.m16n8k16 for 16-bit types:
+//   A (16x16, row):  a0 = (row g,   k 2t..2t+1)  a1 = (row g+8, k 2t..2t+1)
+//                    a2 = (row g,   k 2t+8..9)   a3 = (row g+8, k 2t+8..9)
+//   B (16x8, col):   b0 = (k 2t..2t+1, col g)    b1 = (k 2t+8..9, col g)
+//   C (16x8, f32):   c0,c1 = (row g, cols 2t, 2t+1)  c2,c3 = (row g+8, same)
+// with g = lane / 4 and t = lane % 4; the lower half of each 32-bit register
+// holds the element with the lower index.
+#pragma once
+
+#include <cstdint>
+
+namespace isa_dev {
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+// d += a * b
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t b0,
+                                          const uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// bf16 bit patterns, round to nearest even (finite inputs)
+__device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
+  uint32_t r;
+  asm("{ .reg .b16 h; cvt.rn.bf16.f32 h, %1; mov.b32 %0, {h, h}; }" : "=r"(r) : "f"(x));
+  return static_cast<uint16_t>(r & 0xFFFFu);
+}
+__device__ __forceinline__ float bf16_bits_to_f(uint32_t h) { return __uint_as_float(h << 16); }
+
+}  // namespace isa_dev

@@ -88,7 +88,7 @@ typedef struct isa_shape {
   int32_t k_block;           /* 16, 32, 64 or 128                        */
   int32_t num_groups;        /* G                                        */
   const int32_t* q_offsets;  /* device [G+1] or NULL                     */
-  float scale;               /* logit scale, normally 1/sqrt(d)          */
+  float scale;               /* logit scale > 0, normally 1/sqrt(d)      */
 } isa_shape;
 
 /* Sampling parameters of the fused pipeline calls. */
