@@ -34,6 +34,7 @@
 
 #include "isa_internal.h"
 #include "ptx.cuh"
+#include "tmap.h"
 
 namespace isa_impl {
 namespace {
@@ -577,43 +578,14 @@ __global__ void build_tile_list(const int32_t* off, int G, int N, int q_block, T
   if (t == nt - 1) *count = s_tot[t];
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// [B*H, N, D] bf16 viewed as a 3-D tensor; box = 64 columns x box_rows rows.
-bool make_map(CUtensorMap* m, const void* ptr, int BH, int N, int D, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
-  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
 int launch_d(const AttnLaunch& l, const void* q, const void* k, const void* v, cudaStream_t stream) {
   using Lay = Layout<D>;
   const int BH = l.B * l.H;
   CUtensorMap tq, tk, tv;
   const int kv_rows = l.mode == kAttnDense ? kTileRows : l.Bk;
-  if (!make_map(&tq, q, BH, l.N, D, kTileRows) || !make_map(&tk, k, BH, l.N, D, kv_rows) ||
-      !make_map(&tv, v, BH, l.N, D, kv_rows))
+  if (!make_bf16_map(&tq, q, BH, l.N, D, kTileRows) || !make_bf16_map(&tk, k, BH, l.N, D, kv_rows) ||
+      !make_bf16_map(&tv, v, BH, l.N, D, kv_rows))
     return -1;
   AttnArgs a{};
   a.BH = BH;

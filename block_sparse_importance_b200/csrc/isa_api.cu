@@ -143,7 +143,8 @@ isa_status do_score(isa_context* ctx, const isa_shape* s, const void* q, const v
   l.q = q;
   l.k = k;
   l.mass = mass;
-  l.kbar = reinterpret_cast<float*>(w);
+  l.kbar_hi = reinterpret_cast<uint16_t*>(w);
+  l.kbar_lo = l.kbar_hi + BH * nK * s->head_dim;
   w += round_up(BH * nK * s->head_dim * 4);
   l.centroids = centroids ? centroids : reinterpret_cast<float*>(w);
   w += round_up(BH * s->num_groups * C * s->head_dim * 4);

@@ -65,8 +65,8 @@ struct ScoreLaunch {
   float* mass;
   float* centroids;   // [B,H,G,C,D]
   int32_t* counts;    // [B,H,G,C]
-  float* kbar;        // [B,H,nK,D] scratch
-  float* stats;       // [B,H,G,C,2] scratch
+  uint16_t* kbar_hi;  // [B,H,nK,D] bf16 scratch: key-block means, high part
+  uint16_t* kbar_lo;  // [B,H,nK,D] bf16 scratch: key-block means, low part
   int* status;
   int num_sms;
 };

@@ -7,7 +7,8 @@
 // without reordering tokens.  Key blocks are summarised by their means.
 //
 // Three kernels:
-//   key_means_kernel  kbar_b = mean of the valid rows of key block b (fp32);
+//   key_means_kernel  kbar_b = mean of the valid rows of key block b, stored
+//                     as a bf16 hi + lo pair;
 //   kmeans_kernel     per (batch*head, group): Lloyd's k-means, centroids
 //                     initialised at rows floor(c n / C), `iters` rounds of
 //                     nearest-centroid assignment (squared distance, ties to
@@ -23,21 +24,26 @@
 #include <cstdint>
 
 #include "isa_internal.h"
+#include "mma_sync.cuh"
+#include "ptx.cuh"
+#include "tmap.h"
 
 namespace isa_impl {
 namespace {
 
 constexpr int kScoreThreads = 256;
 constexpr int kChunkRows = 128;
-constexpr int kMassRows = 128;    // centroid rows per mass CTA
-constexpr int kMassBlocks = 64;   // key blocks per smem chunk
 
 __device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float(static_cast<uint32_t>(h) << 16); }
 
 // ------------------------------------------------------------ key means
+// kbar_b = mean of the valid rows of key block b, written as a bf16 hi + lo
+// pair (hi = bf16(kbar), lo = bf16(kbar - hi)) for the tensor-core mass product.
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads) key_means_kernel(const uint16_t* __restrict__ k, int N, int Bk,
-                                                                  int nK, float* __restrict__ kbar) {
+                                                                  int nK, uint16_t* __restrict__ kbar_hi,
+                                                                  uint16_t* __restrict__ kbar_lo) {
+  using namespace isa_dev;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x * (kScoreThreads / 32) + warp;
   const int64_t bh = blockIdx.y;
@@ -63,26 +69,46 @@ __global__ void __launch_bounds__(kScoreThreads) key_means_kernel(const uint16_t
     }
   }
   const float inv = 1.0f / static_cast<float>(r1 - r0);
-  float* o = kbar + (bh * nK + b) * D + lane * PER;
+  const int64_t o = (bh * nK + b) * D + lane * PER;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) o[i] = acc[i] * inv;
+  for (int i = 0; i < PER; ++i) {
+    const float m = acc[i] * inv;
+    const uint16_t hi = bf16_bits_rn(m);
+    kbar_hi[o + i] = hi;
+    kbar_lo[o + i] = bf16_bits_rn(m - bf16_bits_to_f(hi));
+  }
 }
 
 // ---------------------------------------------------------------- k-means
-template <int D>
+// One CTA (8 warps) per (batch*head, group).  Rows stream through shared
+// memory 128 at a time (a group of <= 128 rows is loaded once), rows padded to
+// D + 8 elements so that ldmatrix reads are free of bank conflicts.
+// Assignment: dist_c = |mu_c|^2 - 2 x.mu_c (|x|^2 is common to all c) with the
+// dots on tensor cores: x is exact in bf16 and mu_c is split into bf16
+// hi + lo parts (relative error 2^-18), two mma.sync per 16x8x16 tile.
+// Update: the cluster sums are a one-hot product (assignment^T x) on tensor
+// cores, exact products accumulated in fp32; mu_c = sum_c / n_c.
+template <int D, int NTC>
 __global__ void __launch_bounds__(kScoreThreads) kmeans_kernel(const uint16_t* __restrict__ q, int N, int G,
                                                                int q_block, const int32_t* __restrict__ off, int C,
                                                                int iters, float* __restrict__ centroids,
                                                                int32_t* __restrict__ counts, int* status) {
+  using namespace isa_dev;
+  constexpr int XS = D + 8;            // padded row stride (elements)
+  constexpr int KSTEPS = D / 16;       // k-steps of the dot products
+  constexpr int NTD = D / 64;          // 8-column n-tiles of the sums per warp
   extern __shared__ __align__(16) uint8_t sm[];
-  uint16_t* rows = reinterpret_cast<uint16_t*>(sm);                       // [128][D]
-  float* mu = reinterpret_cast<float*>(sm + kChunkRows * D * 2);           // [C][D]
-  float* sums = mu + C * D;                                                // [C][D]
-  int* cnt = reinterpret_cast<int*>(sums + C * D);                        // [C]
-  int* assign = cnt + 16;                                                  // [128]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(sm);                          // [128][XS]
+  uint16_t* mhi = xs + kChunkRows * XS;                                     // [16][XS]
+  uint16_t* mlo = mhi + 16 * XS;                                            // [16][XS]
+  float* mu = reinterpret_cast<float*>(mlo + 16 * XS);                      // [16][D]
+  float* musq = mu + 16 * D;                                                // [16]
+  int* cnt = reinterpret_cast<int*>(musq + 16);                             // [16]
+  int* assign = cnt + 16;                                                   // [128]
   const int g = blockIdx.x;
   const int64_t bh = blockIdx.y;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, tq = lane & 3;
   int r0, r1;
   if (off) {
     r0 = off[g];
@@ -97,73 +123,148 @@ __global__ void __launch_bounds__(kScoreThreads) kmeans_kernel(const uint16_t* _
   }
   const int n = r1 - r0;
   const uint16_t* qg = q + (bh * N + r0) * D;
-  for (int i = tid; i < C * D; i += kScoreThreads) {
+  for (int i = tid; i < 16 * D; i += kScoreThreads) {
     const int c = i / D, j = i - c * D;
     const int r = static_cast<int>((static_cast<int64_t>(c) * n) / C);
-    mu[i] = n > 0 ? bf16_to_f(qg[static_cast<int64_t>(r) * D + j]) : 0.0f;
+    mu[i] = (c < C && n > 0) ? bf16_to_f(qg[static_cast<int64_t>(r) * D + j]) : 0.0f;
   }
   const bool one_chunk = n <= kChunkRows;
+  const uint32_t xs_base = smem_addr(xs), mhi_base = smem_addr(mhi), mlo_base = smem_addr(mlo);
+  // ldmatrix row address of this lane for a 16x16 A tile at (row0, col0)
+  const int a_row = (lane & 7) + ((lane >> 3) & 1) * 8, a_col = (lane >> 4) * 8;
+  // x2 B tile (8 centroid rows x 16 k): lanes 0-7 k 0-7, lanes 8-15 k 8-15
+  const int b_row = lane & 7, b_col = ((lane >> 3) & 1) * 8;
+  // x4 / x2 trans B tile from x rows: matrices (k 0-7, n 0-7), (k 8-15, n 0-7), (k 0-7, n 8-15), (k 8-15, n 8-15)
+  const int t_row = (lane & 7) + ((lane >> 3) & 1) * 8, t_col = (lane >> 4) * 8;
+  __syncthreads();
   for (int it = 0; it < iters; ++it) {
-    for (int i = tid; i < C * D; i += kScoreThreads) sums[i] = 0.0f;
+    // split the centroids into bf16 hi + lo and take |mu|^2
+    for (int i = tid; i < 16 * D; i += kScoreThreads) {
+      const int c = i / D, j = i - c * D;
+      const float m = mu[i];
+      const uint16_t hi = bf16_bits_rn(m);
+      const uint16_t lo = bf16_bits_rn(m - bf16_bits_to_f(hi));
+      mhi[c * XS + j] = hi;
+      mlo[c * XS + j] = lo;
+    }
+    for (int c = warp; c < 16; c += kScoreThreads / 32) {
+      float acc = 0.0f;
+      for (int j = lane; j < D; j += 32) acc = fmaf(mu[c * D + j], mu[c * D + j], acc);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) musq[c] = acc;
+    }
     if (tid < 16) cnt[tid] = 0;
+    float sums[NTD][4];
+#pragma unroll
+    for (int i = 0; i < NTD; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sums[i][k] = 0.0f;
     __syncthreads();
     for (int cs = 0; cs < n; cs += kChunkRows) {
       const int rc = min(kChunkRows, n - cs);
       if (!(one_chunk && it > 0)) {
-        const uint4* src = reinterpret_cast<const uint4*>(qg + static_cast<int64_t>(cs) * D);
-        uint4* dst = reinterpret_cast<uint4*>(rows);
-        for (int i = tid; i < rc * D / 8; i += kScoreThreads) dst[i] = src[i];
+        // rows [cs, cs+rc) into the padded buffer; rows past rc are zeroed
+        for (int i = tid; i < kChunkRows * (D / 8); i += kScoreThreads) {
+          const int r = i / (D / 8), c16 = i - r * (D / 8);
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (r < rc) v = reinterpret_cast<const uint4*>(qg + static_cast<int64_t>(cs + r) * D)[c16];
+          *reinterpret_cast<uint4*>(xs + r * XS + c16 * 8) = v;
+        }
+        __syncthreads();
       }
-      __syncthreads();
-      // assignment: two threads per row, each summing half of the columns
-      {
-        const int r = tid >> 1, half = tid & 1;
-        int best_c = 0;
-        float best = INFINITY;
-        for (int c = 0; c < C; ++c) {
-          float part = 0.0f;
-          if (r < rc) {
-            const uint16_t* x = rows + r * D + half * (D / 2);
-            const float* m = mu + c * D + half * (D / 2);
-#pragma unroll 16
-            for (int j = 0; j < D / 2; ++j) {
-              const float t = bf16_to_f(x[j]) - m[j];
-              part = fmaf(t, t, part);
+      // ---- assignment: warp w takes rows 16w .. 16w+15
+      if (16 * warp < rc) {
+        float acc[NTC][4];
+#pragma unroll
+        for (int i = 0; i < NTC; ++i)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc[i][k] = 0.0f;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          uint32_t a[4];
+          ldsm_x4(a, xs_base + 2u * ((16 * warp + a_row) * XS + ks * 16 + a_col));
+#pragma unroll
+          for (int nt = 0; nt < NTC; ++nt) {
+            uint32_t bh2[2], bl2[2];
+            const uint32_t off_b = 2u * ((8 * nt + b_row) * XS + ks * 16 + b_col);
+            ldsm_x2(bh2, mhi_base + off_b);
+            ldsm_x2(bl2, mlo_base + off_b);
+            mma_16816(acc[nt], a, bh2[0], bh2[1]);
+            mma_16816(acc[nt], a, bl2[0], bl2[1]);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // rows gq and gq + 8
+          float best = INFINITY;
+          int bi = 0;
+#pragma unroll
+          for (int nt = 0; nt < NTC; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = 8 * nt + 2 * tq + e;
+              const float dist = musq[c] - 2.0f * acc[nt][2 * h + e];
+              if (c < C && dist < best) {
+                best = dist;
+                bi = c;
+              }
+            }
+#pragma unroll
+          for (int o = 1; o <= 2; o <<= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ob < best || (ob == best && oi < bi)) {
+              best = ob;
+              bi = oi;
             }
           }
-          const float dist = part + __shfl_xor_sync(0xffffffffu, part, 1);
-          if (dist < best) {
-            best = dist;
-            best_c = c;
+          const int r = 16 * warp + gq + 8 * h;
+          if (tq == 0) {
+            if (r < rc) {
+              assign[r] = bi;
+              atomicAdd(&cnt[bi], 1);
+            } else {
+              assign[r] = -1;
+            }
           }
         }
-        if (r < rc && half == 0) assign[r] = best_c;
+      } else if (lane < 16) {
+        assign[16 * warp + lane] = -1;
       }
       __syncthreads();
-      // accumulate rows into their cluster sums: thread = (column, half of rows)
-      {
-        constexpr int kColThreads = D;
-        const int j = tid % kColThreads, part = tid / kColThreads, nparts = kScoreThreads / kColThreads;
-        float acc[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) acc[c] = 0.0f;
-        for (int r = part; r < rc; r += nparts) {
-          const float v = bf16_to_f(rows[r * D + j]);
-          const int a = assign[r];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) acc[c] += (a == c) ? v : 0.0f;
+      // ---- cluster sums: one-hot(assign)^T x; warp w owns columns [8 NTD w, 8 NTD (w+1))
+      for (int k0 = 0; k0 < rc; k0 += 16) {
+        uint32_t a[4];
+        const int ka = k0 + 2 * tq, kb = ka + 8;
+        const int s0 = assign[ka], s1 = assign[ka + 1], s2 = assign[kb], s3 = assign[kb + 1];
+        const uint32_t one = 0x3F80u;
+        a[0] = (s0 == gq ? one : 0u) | ((s1 == gq ? one : 0u) << 16);
+        a[1] = (s0 == gq + 8 ? one : 0u) | ((s1 == gq + 8 ? one : 0u) << 16);
+        a[2] = (s2 == gq ? one : 0u) | ((s3 == gq ? one : 0u) << 16);
+        a[3] = (s2 == gq + 8 ? one : 0u) | ((s3 == gq + 8 ? one : 0u) << 16);
+        if constexpr (NTD == 2) {
+          uint32_t b[4];
+          ldsm_x4_trans(b, xs_base + 2u * ((k0 + t_row) * XS + 16 * warp + t_col));
+          mma_16816(sums[0], a, b[0], b[1]);
+          mma_16816(sums[1], a, b[2], b[3]);
+        } else {
+          uint32_t b[2];
+          ldsm_x2_trans(b, xs_base + 2u * ((k0 + (lane & 15)) * XS + 8 * warp));
+          mma_16816(sums[0], a, b[0], b[1]);
         }
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          if (c < C) atomicAdd(&sums[c * D + j], acc[c]);
-        for (int r = tid; r < rc; r += kScoreThreads) atomicAdd(&cnt[assign[r]], 1);
       }
       __syncthreads();
     }
-    for (int i = tid; i < C * D; i += kScoreThreads) {
-      const int c = i / D;
-      if (cnt[c] > 0) mu[i] = sums[i] / static_cast<float>(cnt[c]);
-    }
+    // ---- update: each (cluster, column) is owned by one thread
+#pragma unroll
+    for (int nt = 0; nt < NTD; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = gq + 8 * (e >> 1);
+        const int j = 8 * (NTD * warp + nt) + 2 * tq + (e & 1);
+        const int nc = cnt[c];
+        if (c < C && nc > 0) mu[c * D + j] = sums[nt][e] / static_cast<float>(nc);
+      }
     __syncthreads();
   }
   const int64_t t = bh * G + g;
@@ -171,184 +272,285 @@ __global__ void __launch_bounds__(kScoreThreads) kmeans_kernel(const uint16_t* _
   if (tid < C) counts[t * C + tid] = cnt[tid];
 }
 
+template <int D>
+size_t kmeans_smem_bytes() {
+  constexpr int XS = D + 8;
+  return (kChunkRows * XS + 2 * 16 * XS) * 2 + (16 * D + 16) * 4 + (16 + kChunkRows) * 4;
+}
+
 // ------------------------------------------------------------------ mass
-// Rows of the CTA: group gl (0 .. 128/Cp - 1) owns rows [gl*Cp, gl*Cp + C)
-// with Cp = C rounded up to a power of two; padding rows carry count 0.
-// Thread t: row slab rs = t / 16 (8 rows), block lane bl = t % 16 (4 blocks
-// of each 64-block chunk).
+// One CTA per (batch*head, 128 centroid rows = 128 / Cp groups; Cp = C
+// rounded up to a power of two, padding rows carry weight 0).
+//   logits  l_{c,b} = scale mu_c . kbar_b (+ ln(L_b / Bk) on a partial tail
+//           block; the common ln Bk cancels in the softmax), computed on
+//           tensor cores: mu and kbar are bf16 hi + lo pairs and three
+//           tcgen05.mma products (hi.hi + hi.lo + lo.hi) accumulate in TMEM;
+//   pass 0  each row's online max and sum of exp over all key blocks;
+//   pass 1  the logits again, p = n_c exp(l - max) / sum, summed over the Cp
+//           rows of each group by a reduce-scatter across lanes, and written.
+// Warps 0-3: one thread per centroid row (TMEM lane); warp 4: TMA producer of
+// the kbar tiles (128 blocks x d, hi and lo) into a 2-stage ring; warp 5:
+// MMA issue.  S is double-buffered in TMEM (2 x 128 columns).
+constexpr int kMassThreads = 192;
+constexpr int kMassRing = 2;
+
+template <int D>
+struct MassLayout {
+  static constexpr uint32_t kTile = 128 * D * 2;           // one 128-row bf16 tile
+  static constexpr uint32_t kChunk = 128 * 128;            // 128 rows x 64 bf16
+  static constexpr uint32_t kAHi = 0, kALo = kTile, kRing = 2 * kTile;
+  static constexpr uint32_t kStage = 2 * kTile;            // kbar hi + lo
+  static constexpr uint32_t kBar = kRing + kMassRing * kStage;
+  static constexpr int kBarFull = 0, kBarEmpty = kMassRing, kBarSFull = 2 * kMassRing, kBarSFree = kBarSFull + 2,
+                       kBarFinal = kBarSFree + 2, kNumBars = kBarFinal + 1;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8;
+  static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
+};
+
 template <int D, int Cp>
-__global__ void __launch_bounds__(kScoreThreads) mass_kernel(const float* __restrict__ centroids,
-                                                             const int32_t* __restrict__ counts,
-                                                             const float* __restrict__ kbar, int N, int Bk,
-                                                             int nK, int G, int C, float scale,
-                                                             float* __restrict__ mass) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  constexpr int KP = D + 4;  // padded row stride of the key chunk (floats)
-  float* cen = reinterpret_cast<float*>(sm);               // [128][D]
-  float* kb = cen + kMassRows * D;                          // [64][KP]
-  float* stat_m = kb + kMassBlocks * KP;                    // [128]
-  float* stat_z = stat_m + kMassRows;                       // [128]
-  float* wgt = stat_z + kMassRows;                          // [128] n_c (0 for padding)
-  const int tid = threadIdx.x;
+__global__ void __launch_bounds__(kMassThreads, 1)
+    mass_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
+                const float* __restrict__ centroids, const int32_t* __restrict__ counts, int N, int Bk, int nK,
+                int G, int C, float scale_log2, float* __restrict__ mass, int* status) {
+  using namespace isa_dev;
+  using L = MassLayout<D>;
+  constexpr int kGroupsPerTile = 128 / Cp;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + L::kBar + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t bh = blockIdx.y;
-  const int gpc = kMassRows / Cp;
-  const int g0 = blockIdx.x * gpc;
-  for (int i = tid; i < kMassRows; i += kScoreThreads) {
-    const int gl = i / Cp, c = i - gl * Cp, g = g0 + gl;
-    wgt[i] = (c < C && g < G) ? static_cast<float>(counts[(bh * G + g) * C + c]) : 0.0f;
-  }
-  for (int i = tid; i < kMassRows * D; i += kScoreThreads) {
-    const int rr = i / D, j = i - rr * D;
-    const int gl = rr / Cp, c = rr - gl * Cp, g = g0 + gl;
-    cen[i] = (c < C && g < G) ? centroids[((bh * G + g) * C + c) * D + j] : 0.0f;
-  }
-  const int rs = tid >> 4, bl = tid & 15;
-  float run_m[8], run_z[8];
+  const int g0 = blockIdx.x * kGroupsPerTile;
+  const int T = (nK + 127) / 128;
+  const int n_items = 2 * T;
+
+  // centroid rows -> bf16 hi / lo, K-major with the 128-byte swizzle (16-byte
+  // granule q of row r stored at granule q ^ (r & 7) of the row)
+  for (int i = tid; i < 128 * (D / 8); i += kMassThreads) {
+    const int r = i / (D / 8), q = i - r * (D / 8);
+    const int gl = r / Cp, c = r - gl * Cp, g = g0 + gl;
+    float v[8];
+    if (c < C && g < G) {
+      const float4* src = reinterpret_cast<const float4*>(centroids + ((bh * G + g) * C + c) * D + q * 8);
+      const float4 x0 = src[0], x1 = src[1];
+      v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w; v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+    } else {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    run_m[i] = -INFINITY;
-    run_z[i] = 0.0f;
+      for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+    }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint16_t h0 = bf16_bits_rn(v[2 * e]), h1 = bf16_bits_rn(v[2 * e + 1]);
+      const uint16_t l0 = bf16_bits_rn(v[2 * e] - bf16_bits_to_f(h0));
+      const uint16_t l1 = bf16_bits_rn(v[2 * e + 1] - bf16_bits_to_f(h1));
+      hi[e] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+      lo[e] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+    }
+    const int chunk = q >> 3, qq = q & 7;
+    const uint32_t off = chunk * L::kChunk + r * 128 + ((qq ^ (r & 7)) << 4);
+    *reinterpret_cast<uint4*>(smem + L::kAHi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(smem + L::kALo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
-  const float* kbh = kbar + bh * nK * D;
-  for (int pass = 0; pass < 2; ++pass) {
-    if (pass == 1) {
-      // combine the 16 partial (max, sum) of each row and publish them
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float m = run_m[i], z = run_z[i];
-#pragma unroll
-        for (int o = 1; o < 16; o <<= 1) {
-          const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-          const float z2 = __shfl_xor_sync(0xffffffffu, z, o);
-          const float mm = fmaxf(m, m2);
-          z = (mm == -INFINITY) ? 0.0f : z * __expf(m - mm) + z2 * __expf(m2 - mm);
-          m = mm;
+  if (tid == 0) {
+    for (int i = 0; i < kMassRing; ++i) {
+      mbar_init(bar(L::kBarFull + i), 1);
+      mbar_init(bar(L::kBarEmpty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::kBarSFull + i), 1);
+      mbar_init(bar(L::kBarSFree + i), 128);
+    }
+    mbar_init(bar(L::kBarFinal), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_addr(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  // the generic-proxy stores of the A tiles must be visible to the tensor cores
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    uint32_t issued = 0;
+    bool ok = true;
+    if (lane == 0) {
+      for (int i = 0; i < n_items && ok; ++i) {
+        const uint32_t slot = i % kMassRing, use = i / kMassRing;
+        if (!mbar_wait(bar(L::kBarEmpty + slot), (use & 1u) ^ 1u, abort_flag, kWaitTimeoutNs)) {
+          ok = false;
+          break;
         }
-        if (bl == 0) {
-          stat_m[rs * 8 + i] = m;
-          stat_z[rs * 8 + i] = z;
+        mbar_arrive_expect_tx(bar(L::kBarFull + slot), L::kStage);
+        const uint32_t dst = base + L::kRing + slot * L::kStage;
+        const int row = (i % T) * 128;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(dst + c * L::kChunk, &tm_hi, bar(L::kBarFull + slot), c * 64, row, static_cast<int>(bh));
+          tma_load_3d(dst + L::kTile + c * L::kChunk, &tm_lo, bar(L::kBarFull + slot), c * 64, row,
+                      static_cast<int>(bh));
+        }
+        ++issued;
+      }
+      if (!ok || *abort_flag) {
+        const uint32_t first = issued > kMassRing ? issued - kMassRing : 0;
+        for (uint32_t i = first; i < issued; ++i) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(bar(L::kBarFull + i % kMassRing), (i / kMassRing) & 1u))
+            if (global_timer_ns() - t0 > 200000000ull) break;
         }
       }
     }
-    for (int cb = 0; cb < nK; cb += kMassBlocks) {
-      __syncthreads();
-      for (int i = tid; i < kMassBlocks * D / 4; i += kScoreThreads) {
-        const int b = i / (D / 4), j4 = i - b * (D / 4);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (cb + b < nK) v = reinterpret_cast<const float4*>(kbh + static_cast<int64_t>(cb + b) * D)[j4];
-        float* dst = kb + b * KP + 4 * j4;
-        dst[0] = v.x;
-        dst[1] = v.y;
-        dst[2] = v.z;
-        dst[3] = v.w;
-      }
-      __syncthreads();
-      float acc[8][4];
+  } else if (warp == 5) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0);
+      for (int i = 0; i < n_items; ++i) {
+        const uint32_t slot = i % kMassRing, buf = i & 1;
+        if (!mbar_wait(bar(L::kBarFull + slot), (i / kMassRing) & 1u, abort_flag, kWaitTimeoutNs)) break;
+        if (!mbar_wait(bar(L::kBarSFree + buf), ((i >> 1) & 1u) ^ 1u, abort_flag, kWaitTimeoutNs)) break;
+        tc_fence_after();
+        const uint32_t b_hi = base + L::kRing + slot * L::kStage, b_lo = b_hi + L::kTile;
+        const uint32_t a_hi = base + L::kAHi, a_lo = base + L::kALo;
+        const uint32_t d = tmem + buf * 128;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) acc[i][u] = 0.0f;
-      for (int j = 0; j < D; j += 4) {
-        float4 kv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) kv[u] = *reinterpret_cast<const float4*>(kb + (bl * 4 + u) * KP + j);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 cv = *reinterpret_cast<const float4*>(cen + (rs * 8 + i) * D + j);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            acc[i][u] = fmaf(cv.x, kv[u].x, acc[i][u]);
-            acc[i][u] = fmaf(cv.y, kv[u].y, acc[i][u]);
-            acc[i][u] = fmaf(cv.z, kv[u].z, acc[i][u]);
-            acc[i][u] = fmaf(cv.w, kv[u].w, acc[i][u]);
-          }
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * L::kChunk + (k & 3) * 32;
+          mma_ss(d, smem_desc_sw128(a_hi + off, 16, 1024), smem_desc_sw128(b_hi + off, 16, 1024), idesc,
+                 k > 0 ? 1u : 0u);
+          mma_ss(d, smem_desc_sw128(a_hi + off, 16, 1024), smem_desc_sw128(b_lo + off, 16, 1024), idesc, 1u);
+          mma_ss(d, smem_desc_sw128(a_lo + off, 16, 1024), smem_desc_sw128(b_hi + off, 16, 1024), idesc, 1u);
         }
+        tc_commit(bar(L::kBarEmpty + slot));
+        tc_commit(bar(L::kBarSFull + buf));
       }
-      float lnL[4];
-      bool ok[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int b = cb + bl * 4 + u;
-        ok[u] = b < nK;
-        lnL[u] = ok[u] ? logf(static_cast<float>(min(Bk, N - b * Bk))) : 0.0f;
-      }
+      tc_commit(bar(L::kBarFinal));
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bar(L::kBarFinal), 0))
+        if (global_timer_ns() - t0 > 200000000ull) break;
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int row = tid;  // centroid row == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int gl = row / Cp, c = row - gl * Cp, g = g0 + gl;
+    const float n_c = (c < C && g < G) ? static_cast<float>(counts[(bh * G + g) * C + c]) : 0.0f;
+    const int tail_rows = N - (nK - 1) * Bk;
+    const float tail_adj = tail_rows < Bk ? log2f(static_cast<float>(tail_rows) / static_cast<float>(Bk)) : 0.0f;
+    float m_run = -INFINITY, z_run = 0.0f, w = 0.0f;
+    constexpr int kCols = 32 / Cp;  // columns a lane owns after the reduce-scatter of a 32-column chunk
+    for (int i = 0; i < n_items; ++i) {
+      const int pass = i / T, j = i - pass * T;
+      const uint32_t buf = i & 1;
+      if (!mbar_wait(bar(L::kBarSFull + buf), (i >> 1) & 1u, abort_flag, kWaitTimeoutNs)) break;
+      tc_fence_after();
+      const int col0 = j * 128;
       if (pass == 0) {
+        float tmax = -INFINITY;
+        float zs[4][32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t sv[32];
+          tmem_ld32(lane_base + buf * 128 + 32 * cc, sv);
+          tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (!ok[u]) continue;
-            const float l = fmaf(scale, acc[i][u], lnL[u]);
-            if (l > run_m[i]) {
-              run_z[i] = run_z[i] * __expf(run_m[i] - l) + 1.0f;
-              run_m[i] = l;
-            } else {
-              run_z[i] += __expf(l - run_m[i]);
-            }
+          for (int e = 0; e < 32; ++e) {
+            const int b = col0 + 32 * cc + e;
+            float z = __uint_as_float(sv[e]) * scale_log2;
+            if (b == nK - 1) z += tail_adj;
+            z = b < nK ? z : -INFINITY;
+            zs[cc][e] = z;
+            tmax = fmaxf(tmax, z);
           }
         }
+        const float m_new = fmaxf(m_run, tmax);
+        float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) part[e & 3] += fast_exp2(zs[cc][e] - m_new);
+        z_run = (m_run == -INFINITY ? 0.0f : z_run * fast_exp2(m_run - m_new)) + ((part[0] + part[1]) + (part[2] + part[3]));
+        m_run = m_new;
+        if (j == T - 1) w = z_run > 0.0f ? n_c / z_run : 0.0f;
       } else {
-        // rows of this thread: 8 consecutive rows = 8/Cp whole groups (Cp <= 8)
-        // or half of a 16-row group (Cp == 16, combined with the partner slab)
-        float part[4][8];
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t sv[32];
+          tmem_ld32(lane_base + buf * 128 + 32 * cc, sv);
+          tmem_wait_ld();
+          float v[32];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) part[u][i] = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = rs * 8 + i;
-          const float w = wgt[rr];
-          const float m = stat_m[rr], z = stat_z[rr];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float l = fmaf(scale, acc[i][u], lnL[u]);
-            part[u][i] = (w > 0.0f && ok[u]) ? w * (__expf(l - m) / z) : 0.0f;
+          for (int e = 0; e < 32; ++e) {
+            const int b = col0 + 32 * cc + e;
+            float z = __uint_as_float(sv[e]) * scale_log2;
+            if (b == nK - 1) z += tail_adj;
+            v[e] = b < nK ? w * fast_exp2(z - m_run) : 0.0f;
           }
-        }
-        if constexpr (Cp <= 8) {
+          // reduce-scatter over the Cp rows of each group: lane p of a group
+          // ends with the group's sums for columns [p * kCols, (p+1) * kCols)
 #pragma unroll
-          for (int s0 = 0; s0 < 8; s0 += Cp) {
-            const int gl = (rs * 8 + s0) / Cp, g = g0 + gl;
+          for (int m = Cp / 2, cnt = 16; m >= 1; m >>= 1, cnt >>= 1) {
+            const bool up = (lane & m) != 0;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              float sum = 0.0f;
-#pragma unroll
-              for (int i = s0; i < s0 + Cp; ++i) sum += part[u][i];
-              const int b = cb + bl * 4 + u;
-              if (g < G && ok[u]) mass[(bh * G + g) * nK + b] = sum;
+            for (int e = 0; e < 16; ++e) {
+              if (e < cnt) {
+                const float mine = up ? v[cnt + e] : v[e];
+                const float other = up ? v[e] : v[cnt + e];
+                v[e] = mine + __shfl_xor_sync(0xffffffffu, other, m);
+              }
             }
           }
-        } else {
+          const int p = lane & (Cp - 1);
+          if (g < G) {
+            float* dst = mass + (bh * G + g) * nK;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            float sum = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) sum += part[u][i];
-            sum += __shfl_xor_sync(0xffffffffu, sum, 16);
-            const int gl = (rs * 8) / 16, g = g0 + gl, b = cb + bl * 4 + u;
-            if ((rs & 1) == 0 && g < G && ok[u]) mass[(bh * G + g) * nK + b] = sum;
+            for (int e = 0; e < kCols; ++e) {
+              const int b = col0 + 32 * cc + p * kCols + e;
+              if (b < nK) dst[b] = v[e];
+            }
           }
         }
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarSFree + buf));
     }
-    __syncthreads();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort_flag) atomicCAS(status, 0, kStatusTimeout);
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
   }
 }
 
 template <int D, int Cp>
 int launch_mass(const ScoreLaunch& s, int nK, int BH, cudaStream_t stream) {
-  constexpr int gpc = kMassRows / Cp;
-  const size_t ms_smem = (kMassRows * D + kMassBlocks * (D + 4) + 3 * kMassRows) * 4;
-  static bool ms_attr = false;
-  if (!ms_attr) {
+  using L = MassLayout<D>;
+  CUtensorMap thi, tlo;
+  if (!make_bf16_map(&thi, s.kbar_hi, BH, nK, D, 128) || !make_bf16_map(&tlo, s.kbar_lo, BH, nK, D, 128)) return -1;
+  static bool attr = false;
+  if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(mass_kernel<D, Cp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(ms_smem));
+                                         static_cast<int>(L::kAlloc));
     if (e != cudaSuccess) return static_cast<int>(e);
-    ms_attr = true;
+    attr = true;
   }
-  mass_kernel<D, Cp><<<dim3((s.G + gpc - 1) / gpc, BH), kScoreThreads, ms_smem, stream>>>(
-      s.centroids, s.counts, s.kbar, s.N, s.Bk, nK, s.G, s.C, s.scale, s.mass);
+  constexpr int gpt = 128 / Cp;
+  mass_kernel<D, Cp><<<dim3((s.G + gpt - 1) / gpt, BH), kMassThreads, L::kAlloc, stream>>>(
+      thi, tlo, s.centroids, s.counts, s.N, s.Bk, nK, s.G, s.C, s.scale * 1.4426950408889634f, s.mass, s.status);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -357,19 +559,27 @@ int launch_score_d(const ScoreLaunch& s, cudaStream_t stream) {
   const int BH = s.B * s.H;
   const int nK = (s.N + s.Bk - 1) / s.Bk;
   key_means_kernel<D><<<dim3((nK + 7) / 8, BH), kScoreThreads, 0, stream>>>(static_cast<const uint16_t*>(s.k), s.N,
-                                                                            s.Bk, nK, s.kbar);
+                                                                            s.Bk, nK, s.kbar_hi, s.kbar_lo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
-  const size_t km_smem = kChunkRows * D * 2 + 2 * s.C * D * 4 + (16 + kChunkRows) * 4;
+  const size_t km_smem = kmeans_smem_bytes<D>();
   static bool km_attr = false;
   if (!km_attr) {
-    e = cudaFuncSetAttribute(kmeans_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024 + 16 * 1024);
+    e = cudaFuncSetAttribute(kmeans_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(km_smem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kmeans_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(km_smem));
     if (e != cudaSuccess) return static_cast<int>(e);
     km_attr = true;
   }
-  kmeans_kernel<D><<<dim3(s.G, BH), kScoreThreads, km_smem, stream>>>(static_cast<const uint16_t*>(s.q), s.N, s.G,
-                                                                      s.q_block, s.q_offsets, s.C, s.iters,
-                                                                      s.centroids, s.counts, s.status);
+  if (s.C <= 8)
+    kmeans_kernel<D, 1><<<dim3(s.G, BH), kScoreThreads, km_smem, stream>>>(
+        static_cast<const uint16_t*>(s.q), s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids, s.counts,
+        s.status);
+  else
+    kmeans_kernel<D, 2><<<dim3(s.G, BH), kScoreThreads, km_smem, stream>>>(
+        static_cast<const uint16_t*>(s.q), s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids, s.counts,
+        s.status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
   int Cp = 1;
