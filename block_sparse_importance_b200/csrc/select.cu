@@ -21,6 +21,8 @@
 //     (i + U 2^-32) T / n' below x is q + [r 2^32 > U T]; block j is drawn
 //     when that count steps between W_{j-1} and W_j;
 //   * drawn blocks get log_w = ln T - ln(n' w) (fp64, stored fp32).
+// Rows of up to 2048 blocks go to a warp-per-row kernel; longer rows to a
+// CTA-per-row kernel.  Both produce identical plans.
 
 #include <cstdint>
 
@@ -298,9 +300,241 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Warp-per-row variant for rows of at most 32 * VPL blocks: lane l holds the
+// contiguous blocks [l*VPL, (l+1)*VPL) in registers, so every scan is a local
+// prefix plus one warp shuffle scan and no block-wide barrier is needed.  The
+// exact set's threshold is found by a bitwise binary search on the keys (the
+// largest t with #{key >= t} >= n_exact).  Same integer arithmetic and same
+// results as select_kernel.
+constexpr int kWarpRowsPerCta = 8;
+
+__device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+// exclusive prefix over lanes
+__device__ __forceinline__ uint64_t warp_excl_u64(uint64_t v, int lane) {
+  uint64_t inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  return inc - v;
+}
+__device__ __forceinline__ uint32_t warp_excl_u32(uint32_t v, int lane) {
+  uint32_t inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  return inc - v;
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(SelectLaunch a) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarpRowsPerCta + warp;
+  const int64_t rows = static_cast<int64_t>(a.B) * a.H * a.G;
+  if (row >= rows) return;
+  const int nK = a.nK;
+  // this warp's shared slice, skewed by one word per 32 so that the blocked
+  // per-lane reads are free of bank conflicts: first the mass row, then the
+  // integer weights of the rest
+  uint32_t* st = reinterpret_cast<uint32_t*>(sm) + warp * (32 * VPL + VPL);
+  auto at = [](int i) { return i + (i >> 5); };
+  const float* m = a.mass + row * nK;
+  for (int i = lane; i < nK; i += 32) st[at(i)] = __float_as_uint(m[i]);
+  __syncwarp();
+  const int g = static_cast<int>(row % a.G);
+  const int h = static_cast<int>((row / a.G) % a.H);
+  const int b = static_cast<int>(row / (static_cast<int64_t>(a.G) * a.H));
+  const int base = lane * VPL;
+  const int nv = max(0, min(VPL, nK - base));  // blocks this lane holds
+  uint32_t key[VPL];
+  bool bad = false;
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    uint32_t k = 0;
+    if (v < nv) {
+      const float x = __uint_as_float(st[at(base + v)]);
+      if (!isfinite(x)) {
+        bad = true;
+      } else if (x > 0.0f) {
+        k = __float_as_uint(x);
+      }
+    }
+    key[v] = k;  // blocks past the row are 0 and never counted (v >= nv)
+  }
+  const int S = a.n_exact + a.n_sample;
+  // ---- exact set: threshold t = largest key with #{key >= t} >= n_exact
+  uint64_t ex = 0;  // bit v: block base+v is exact
+  if (a.n_exact > 0) {
+    uint32_t t = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = t | (1u << bit);
+      uint32_t c = 0;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) c += (v < nv && key[v] >= cand) ? 1u : 0u;
+      if (__reduce_add_sync(0xffffffffu, c) >= static_cast<uint32_t>(a.n_exact)) t = cand;
+    }
+    uint32_t gt = 0, eq = 0;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      gt += (v < nv && key[v] > t) ? 1u : 0u;
+      eq += (v < nv && key[v] == t) ? 1u : 0u;
+    }
+    const uint32_t need = static_cast<uint32_t>(a.n_exact) - __reduce_add_sync(0xffffffffu, gt);
+    uint32_t rank = warp_excl_u32(eq, lane);
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      if (v < nv) {
+        const bool tie = key[v] == t;
+        if (key[v] > t || (tie && rank < need)) ex |= 1ull << v;
+        rank += tie ? 1u : 0u;
+      }
+    }
+  }
+  // ---- the rest: weights (into the shared slice), capping, systematic PPS
+  const int n_rest = nK - a.n_exact;
+  uint64_t cap = 0, drawn = 0;  // bit v: capped (or taken whole), drawn
+  uint64_t T = 0;
+  int n_left = 0;
+  if (a.n_sample >= n_rest) {
+    for (int v = 0; v < nv; ++v)
+      if (!((ex >> v) & 1)) cap |= 1ull << v;
+  } else if (a.n_sample > 0) {
+    uint32_t kmax = 0;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
+      if (v < nv && !((ex >> v) & 1)) kmax = max(kmax, key[v]);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    const double mmax = static_cast<double>(__uint_as_float(kmax));
+    __syncwarp();
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      if (v < nv) {
+        uint32_t wv = 0;
+        if (!((ex >> v) & 1))
+          wv = mmax > 0.0 ? static_cast<uint32_t>(floor(static_cast<double>(__uint_as_float(key[v])) / mmax *
+                                                       2147483648.0)) + 1u
+                          : 1u;
+        st[at(base + v)] = wv;  // 0 marks exact blocks
+      }
+    }
+    int n_capped = 0;
+    for (;;) {
+      uint64_t tl = 0;
+      for (int v = 0; v < nv; ++v)
+        if (!((cap >> v) & 1)) tl += st[at(base + v)];
+      T = warp_sum_u64(tl);
+      n_left = a.n_sample - n_capped;
+      uint32_t add = 0;
+      uint64_t newcap = 0;
+      for (int v = 0; v < nv; ++v) {
+        const uint32_t wv = st[at(base + v)];
+        if (wv != 0 && !((cap >> v) & 1) && static_cast<uint64_t>(n_left) * wv >= T) {
+          newcap |= 1ull << v;
+          ++add;
+        }
+      }
+      const uint32_t add_all = __reduce_add_sync(0xffffffffu, add);
+      if (add_all == 0) break;
+      cap |= newcap;
+      n_capped += static_cast<int>(add_all);
+    }
+    if (n_left > 0) {
+      const uint32_t U = static_cast<uint32_t>(
+          philox_word0(static_cast<uint32_t>(g), static_cast<uint32_t>(h), static_cast<uint32_t>(b), 0, a.seed, 0) >>
+          32);
+      const uint64_t nl = static_cast<uint64_t>(n_left);
+      const uint64_t ut_lo = static_cast<uint64_t>(U) * T;  // U T < 2^76
+      const uint64_t ut_hi = __umul64hi(static_cast<uint64_t>(U), T);
+      // points of the comb below x: q + [r 2^32 > U T] with q = floor(x n' / T)
+      // and r = x n' - q T.  Walking x up by an uncapped weight (n' w < T)
+      // moves r up by n' w and needs at most one reduction by T, so only the
+      // start of each lane's segment takes a division.
+      auto above = [&](uint64_t r_) -> bool {
+        const uint64_t r_hi = r_ >> 32, r_lo = r_ << 32;
+        return r_hi > ut_hi || (r_hi == ut_hi && r_lo > ut_lo);
+      };
+      uint64_t local = 0;
+      for (int v = 0; v < nv; ++v)
+        if (!((cap >> v) & 1)) local += st[at(base + v)];
+      const uint64_t xn0 = warp_excl_u64(local, lane) * nl;
+      uint64_t q = xn0 / T, r = xn0 - q * T;
+      uint64_t f_prev = q + (above(r) ? 1u : 0u);
+      for (int v = 0; v < nv; ++v) {
+        const uint32_t wv = st[at(base + v)];
+        if (wv != 0 && !((cap >> v) & 1)) {
+          r += static_cast<uint64_t>(wv) * nl;
+          if (r >= T) {
+            r -= T;
+            ++q;
+          }
+          const uint64_t f = q + (above(r) ? 1u : 0u);
+          if (f != f_prev) drawn |= 1ull << v;
+          f_prev = f;
+        }
+      }
+    }
+  }
+  // ---- write the plan row: exact ascending, then capped + drawn ascending
+  int32_t* out_idx = a.idx + row * S;
+  float* out_lw = a.log_w + row * S;
+  const uint32_t ne = __popcll(ex), nr = __popcll(cap | drawn);
+  uint32_t pe = warp_excl_u32(ne, lane);
+  uint32_t pr = static_cast<uint32_t>(a.n_exact) + warp_excl_u32(nr, lane);
+  const double lnT = T > 0 ? log(static_cast<double>(T)) : 0.0;
+  for (int v = 0; v < nv; ++v) {
+    const int i = base + v;
+    if ((ex >> v) & 1) {
+      if (pe < static_cast<uint32_t>(a.n_exact)) {
+        out_idx[pe] = i;
+        out_lw[pe] = 0.0f;
+      }
+      ++pe;
+    } else if (((cap | drawn) >> v) & 1) {
+      if (pr < static_cast<uint32_t>(S)) {
+        out_idx[pr] = i;
+        out_lw[pr] = ((drawn >> v) & 1) ? static_cast<float>(lnT - log(static_cast<double>(
+                                                                        static_cast<uint64_t>(n_left) * st[at(i)])))
+                                        : 0.0f;
+      }
+      ++pr;
+    }
+  }
+  const uint32_t tot_e = __reduce_add_sync(0xffffffffu, ne), tot_r = __reduce_add_sync(0xffffffffu, nr);
+  const bool any_bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0 && (any_bad || tot_e != static_cast<uint32_t>(a.n_exact) || tot_e + tot_r != static_cast<uint32_t>(S)))
+    atomicCAS(a.status, 0, kStatusDeviceCheck);
+}
+
+template <int VPL>
+int launch_select_warp(const SelectLaunch& s, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(s.B) * s.H * s.G;
+  const size_t smem = static_cast<size_t>(kWarpRowsPerCta) * (32 * VPL + VPL) * 4;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(select_warp_kernel<VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  const unsigned grid = static_cast<unsigned>((rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta);
+  select_warp_kernel<VPL><<<grid, 32 * kWarpRowsPerCta, smem, stream>>>(s);
+  return static_cast<int>(cudaGetLastError());
+}
+
 }  // namespace
 
 int launch_select(const SelectLaunch& s, cudaStream_t stream) {
+  if (s.nK <= 32 * 8) return launch_select_warp<8>(s, stream);
+  if (s.nK <= 32 * 16) return launch_select_warp<16>(s, stream);
+  if (s.nK <= 32 * 40) return launch_select_warp<40>(s, stream);
+  if (s.nK <= 32 * 64) return launch_select_warp<64>(s, stream);
   const size_t smem = static_cast<size_t>(s.nK) * 9 + 16;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
