@@ -94,6 +94,14 @@ struct Work {
   int bh, g, row0, nrows;
 };
 
+// max of 16 consecutive fp32 values held as raw bits, by 3-input max
+__device__ __forceinline__ float max16(const uint32_t* v) {
+  auto f = [&](int i) { return __uint_as_float(v[i]); };
+  const float m0 = fmax3f(f(0), f(1), f(2)), m1 = fmax3f(f(3), f(4), f(5)), m2 = fmax3f(f(6), f(7), f(8));
+  const float m3 = fmax3f(f(9), f(10), f(11)), m4 = fmax3f(f(12), f(13), f(14));
+  return fmaxf(fmax3f(m0, m1, m2), fmax3f(m3, m4, f(15)));
+}
+
 __device__ __forceinline__ bool decode_work(const AttnArgs& a, int tph, int n_work, int w, Work& r) {
   if (w >= n_work) return false;
   r.bh = w / tph;
@@ -360,28 +368,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!decode_work(a, tph, n_work, 2 * p + x, w)) continue;
       const int64_t prow = (static_cast<int64_t>(w.bh) * a.G + w.g) * a.S;
       float m_used = 0.0f, l_sum = 0.0f;
-      for (int j = 0; j < T; ++j) {
-        // per 16-column chunk of this KV tile: log-weight (log2 units) and
-        // number of valid key rows; lanes 0..7 each work out one chunk
-        float c_bias = 0.0f;
-        int c_valid = 0;
-        if (lane < 8) {
-          const int pos = j * kTileRows + lane * 16;
-          if (dense) {
-            c_valid = max(0, min(16, a.N - pos));
-          } else {
-            const int s = pos / a.Bk;
-            const int within = pos - s * a.Bk;
-            if (s < a.S) {
-              const int b = a.idx[prow + s];
-              if (b >= 0 && b < a.nK) {
-                const int rows = min(a.Bk, a.N - b * a.Bk);
-                c_valid = max(0, min(16, rows - within));
-                c_bias = a.log_w[prow + s] * kLog2e;
-              }
-            }
+      // per 16-column chunk of a KV tile: log-weight (log2 units) and number
+      // of valid key rows; lanes 0..7 each work out one chunk.  The plan's
+      // entries for tile j+1 are loaded while tile j runs and only decoded in
+      // the next iteration, so their latency stays off the critical path.
+      auto fetch = [&](int jj, int& rb, float& rlw) {
+        rb = -1;
+        rlw = 0.0f;
+        if (!dense && lane < 8) {
+          const int s = (jj * kTileRows + lane * 16) / a.Bk;
+          if (s < a.S) {
+            rb = a.idx[prow + s];
+            rlw = a.log_w[prow + s];
           }
         }
+      };
+      auto decode = [&](int jj, int rb, float rlw, float& bias_o, int& valid_o) {
+        bias_o = 0.0f;
+        valid_o = 0;
+        if (lane < 8) {
+          const int pos = jj * kTileRows + lane * 16;
+          if (dense) {
+            valid_o = max(0, min(16, a.N - pos));
+          } else if (rb >= 0 && rb < a.nK) {
+            const int within = pos - (pos / a.Bk) * a.Bk;
+            valid_o = max(0, min(16, min(a.Bk, a.N - rb * a.Bk) - within));
+            bias_o = rlw * kLog2e;
+          }
+        }
+      };
+      int nb_idx;
+      float nb_lw;
+      fetch(0, nb_idx, nb_lw);
+      for (int j = 0; j < T; ++j) {
+        const int cur_idx = nb_idx;
+        const float cur_lw = nb_lw;
+        if (j + 1 < T) fetch(j + 1, nb_idx, nb_lw);
+        float c_bias;
+        int c_valid;
+        decode(j, cur_idx, cur_lw, c_bias, c_valid);
         if (!mbar_wait(bar(L::kBarSFull + x), s_waits & 1u, abort_flag, a.timeout)) {
           ok = false;
           break;
@@ -394,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool partial = __any_sync(0xffffffffu, c_valid > 0 && c_valid < 16);
         // pass 1: row max of z = scale*s + log_w (log2 units) over valid keys.
         // scale > 0, so the max of z over a 16-column chunk is scale * (max of
-        // s) + bias; eight independent accumulators keep the chain short, and
+        // s) + bias; a tree of 3-input maxima keeps the chain short, and
         // the next chunk's TMEM load is in flight while this one is reduced.
         float mx = -INFINITY;
         {
@@ -409,16 +434,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float b1 = __shfl_sync(0xffffffffu, c_bias, 2 * c + 1);
             float h[2];
             if (!partial) {
-              float l4[4], h4[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                l4[i] = fmaxf(fmaxf(__uint_as_float(v[i]), __uint_as_float(v[i + 4])),
-                              fmaxf(__uint_as_float(v[i + 8]), __uint_as_float(v[i + 12])));
-                h4[i] = fmaxf(fmaxf(__uint_as_float(v[16 + i]), __uint_as_float(v[20 + i])),
-                              fmaxf(__uint_as_float(v[24 + i]), __uint_as_float(v[28 + i])));
-              }
-              h[0] = fmaxf(fmaxf(l4[0], l4[1]), fmaxf(l4[2], l4[3]));
-              h[1] = fmaxf(fmaxf(h4[0], h4[1]), fmaxf(h4[2], h4[3]));
+              h[0] = max16(v);
+              h[1] = max16(v + 16);
             } else {
               const int n0 = __shfl_sync(0xffffffffu, c_valid, 2 * c), n1 = __shfl_sync(0xffffffffu, c_valid, 2 * c + 1);
               h[0] = -INFINITY;
