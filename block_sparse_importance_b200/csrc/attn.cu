@@ -43,9 +43,12 @@ using namespace isa_dev;
 
 constexpr int kTileRows = 128;
 constexpr int kRing = 4;
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+// 18 warps: 0-7 softmax of tile A and 8-15 of tile B (in each, warps 0-3
+// take S columns 0-63 and warps 4-7 columns 64-127 of the same 128 rows),
+// 16 TMA producer, 17 MMA issue.
+constexpr int kThreads = 576;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -82,9 +85,12 @@ struct Layout {
   static constexpr int kBarQFull = 0, kBarQEmpty = 2, kBarKVFull = 4, kBarKVEmpty = 4 + kRing,
                        kBarSFull = 4 + 2 * kRing, kBarPFull = kBarSFull + 2,
                        kBarODone = kBarPFull + 2, kBarFinal = kBarODone + 2, kBarStall = kBarFinal + 1,
-                       kNumBars = kBarStall + 1;
+                       kBarXchg = kBarStall + 1, kNumBars = kBarXchg + 8;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr uint32_t kTotal = kMiscOff + 16;
+  // row max and row sum exchange between the two column halves:
+  // [max | sum][tile][half][row]
+  static constexpr uint32_t kXchgOff = kMiscOff + 16;
+  static constexpr uint32_t kTotal = kXchgOff + 2 * 2 * 2 * 128 * 4;
   static constexpr uint32_t kAlloc = kTotal + 1024;
   // TMEM columns
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
@@ -179,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(L::kBarQFull + i), 1);
       mbar_init(bar(L::kBarQEmpty + i), 1);
       mbar_init(bar(L::kBarSFull + i), 1);
-      mbar_init(bar(L::kBarPFull + i), 128);
+      mbar_init(bar(L::kBarPFull + i), 256);
       mbar_init(bar(L::kBarODone + i), 1);
     }
     for (int i = 0; i < kRing; ++i) {
@@ -188,6 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(L::kBarFinal), 1);
     mbar_init(bar(L::kBarStall), 1);  // never arrived at: only the failure-detection hook waits on it
+    for (int i = 0; i < 8; ++i) mbar_init(bar(L::kBarXchg + i), 64);
     *abort_flag = 0;
     *bad_index = 0;
     fence_mbar_init();
@@ -341,7 +348,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t d_o = tmem + (side ? L::kColO1 : L::kColO0);
 #pragma unroll
             for (int k = 0; k < kTileRows / 16; ++k) {
-              mma_ts(d_o, a_p + k * 8, smem_desc_sw128(kv + k * 2048, L::kChunkBytes, 1024), idesc_pv,
+              // keys 0-63: P of the first column half at columns 0-31 of S;
+              // keys 64-127: the second half's P at columns 64-95
+              const uint32_t pcol = k < 4 ? 8 * k : 64 + 8 * (k - 4);
+              mma_ts(d_o, a_p + pcol, smem_desc_sw128(kv + k * 2048, L::kChunkBytes, 1024), idesc_pv,
                      (j > 0 || k > 0) ? 1u : 0u);
             }
             if (j == T - 1) tc_commit(bar(L::kBarODone + side));
@@ -354,29 +364,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(bar(L::kBarFinal));
       drain_wait(bar(L::kBarFinal), 0);
     }
-  } else if (warp < 8) {
+  } else if (warp < 16) {
     // ------------------------------------------------------------- softmax
-    const int x = warp >> 2;            // which tile of the pair
-    const int row = tid & 127;          // row of the tile == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t col_s = x ? L::kColS1 : L::kColS0;
-    const uint32_t col_o = x ? L::kColO1 : L::kColO0;
-    uint32_t s_waits = 0, o_waits = 0;
+    // one thread per (row, column half): row = TMEM lane, the half's 64
+    // columns of S and D/2 columns of O
+    const int x = warp >> 3;            // which tile of the pair
+    const int hf = (warp >> 2) & 1;     // column half
+    const int q4 = warp & 3;            // TMEM lane quarter
+    const int row = q4 * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint32_t col_s = (x ? L::kColS1 : L::kColS0) + 64 * hf;  // this half's S; its P lands here too
+    const uint32_t col_o = (x ? L::kColO1 : L::kColO0) + (D / 2) * hf;
+    // separate max and sum slots: a half rewrites a slot only after its partner
+    // has passed the read of the previous value (the next S needs the
+    // partner's P, and the epilogue needs all of it)
+    float* xchg_max = reinterpret_cast<float*>(smem + L::kXchgOff) + x * 256;        // [half][row]
+    float* xchg_sum = reinterpret_cast<float*>(smem + L::kXchgOff) + 512 + x * 256;  // [half][row]
+    const uint32_t xbar = bar(L::kBarXchg + x * 4 + q4);
+    uint32_t s_waits = 0, o_waits = 0, x_waits = 0;
     bool ok = true;
+    // combine a per-row value with the other half's (bounded wait on the pair's barrier)
+    auto exchange = [&](float v, bool is_max, float& out) -> bool {
+      float* xchg = is_max ? xchg_max : xchg_sum;
+      xchg[hf * 128 + row] = v;
+      mbar_arrive(xbar);
+      if (!mbar_wait(xbar, x_waits & 1u, abort_flag, a.timeout)) return false;
+      ++x_waits;
+      const float o = xchg[(1 - hf) * 128 + row];
+      out = is_max ? fmaxf(v, o) : v + o;
+      return true;
+    };
     for (int p = blockIdx.x; p < n_pairs && ok; p += gridDim.x) {
       Work w;
       if (!decode_work(a, tph, n_work, 2 * p + x, w)) continue;
       const int64_t prow = (static_cast<int64_t>(w.bh) * a.G + w.g) * a.S;
       float m_used = 0.0f, l_sum = 0.0f;
-      // per 16-column chunk of a KV tile: log-weight (log2 units) and number
-      // of valid key rows; lanes 0..7 each work out one chunk.  The plan's
-      // entries for tile j+1 are loaded while tile j runs and only decoded in
-      // the next iteration, so their latency stays off the critical path.
+      // per 16-column chunk of this half: log-weight (log2 units) and number of
+      // valid key rows; lanes 0..3 each work out one chunk.  The plan's entries
+      // for tile j+1 are loaded while tile j runs and decoded a tile later.
       auto fetch = [&](int jj, int& rb, float& rlw) {
         rb = -1;
         rlw = 0.0f;
-        if (!dense && lane < 8) {
-          const int s = (jj * kTileRows + lane * 16) / a.Bk;
+        if (!dense && lane < 4) {
+          const int s = (jj * kTileRows + 64 * hf + lane * 16) / a.Bk;
           if (s < a.S) {
             rb = a.idx[prow + s];
             rlw = a.log_w[prow + s];
@@ -386,8 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto decode = [&](int jj, int rb, float rlw, float& bias_o, int& valid_o) {
         bias_o = 0.0f;
         valid_o = 0;
-        if (lane < 8) {
-          const int pos = jj * kTileRows + lane * 16;
+        if (lane < 4) {
+          const int pos = jj * kTileRows + 64 * hf + lane * 16;
           if (dense) {
             valid_o = max(0, min(16, a.N - pos));
           } else if (rb >= 0 && rb < a.nK) {
@@ -417,49 +447,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         // sequence (a partial tail block) needs per-element masking
         if (c_valid == 0) c_bias = -INFINITY;
         const bool partial = __any_sync(0xffffffffu, c_valid > 0 && c_valid < 16);
-        // pass 1: row max of z = scale*s + log_w (log2 units) over valid keys.
-        // scale > 0, so the max of z over a 16-column chunk is scale * (max of
-        // s) + bias; a tree of 3-input maxima keeps the chain short, and
-        // the next chunk's TMEM load is in flight while this one is reduced.
+        // pass 1: this half's row max of z = scale*s + log_w (log2 units);
+        // scale > 0, so a chunk's max is scale * (max of s) + its bias
         float mx = -INFINITY;
         {
-          uint32_t sv[2][32];
-          tmem_ld32(lane_base + col_s, sv[0]);
+          uint32_t sv[2][16];
+          tmem_ld16(lane_base + col_s, sv[0]);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            if (c < 3) tmem_ld32(lane_base + col_s + 32 * (c + 1), sv[(c + 1) & 1]);
+            if (c < 3) tmem_ld16(lane_base + col_s + 16 * (c + 1), sv[(c + 1) & 1]);
             const uint32_t* v = sv[c & 1];
-            const float b0 = __shfl_sync(0xffffffffu, c_bias, 2 * c);
-            const float b1 = __shfl_sync(0xffffffffu, c_bias, 2 * c + 1);
-            float h[2];
+            const float bias = __shfl_sync(0xffffffffu, c_bias, c);
+            float hm;
             if (!partial) {
-              h[0] = max16(v);
-              h[1] = max16(v + 16);
+              hm = max16(v);
             } else {
-              const int n0 = __shfl_sync(0xffffffffu, c_valid, 2 * c), n1 = __shfl_sync(0xffffffffu, c_valid, 2 * c + 1);
-              h[0] = -INFINITY;
-              h[1] = -INFINITY;
+              const int nv = __shfl_sync(0xffffffffu, c_valid, c);
+              hm = -INFINITY;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const bool ok_i = (i & 15) < (i < 16 ? n0 : n1);
-                if (ok_i) h[i >> 4] = fmaxf(h[i >> 4], __uint_as_float(v[i]));
-              }
+              for (int i = 0; i < 16; ++i)
+                if (i < nv) hm = fmaxf(hm, __uint_as_float(v[i]));
             }
-            mx = fmaxf(mx, fmaxf(fmaf(h[0], a.scale_log2, b0), fmaf(h[1], a.scale_log2, b1)));
+            mx = fmaxf(mx, fmaf(hm, a.scale_log2, bias));
             if (c < 3) tmem_wait_ld();
           }
+        }
+        if (!exchange(mx, true, mx)) {
+          ok = false;
+          break;
         }
         if (j == 0) {
           m_used = mx == -INFINITY ? 0.0f : mx;
         } else if (__any_sync(0xffffffffu, mx > m_used + kRescaleLog2)) {
-          // raise the running max and rescale this row's O and sum in place
+          // raise the running max and rescale this half's O columns and sum
           const float m_new = fmaxf(m_used, mx);
           const float f = fast_exp2(m_used - m_new);
           m_used = m_new;
           l_sum *= f;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < D / 64; ++c) {
             uint32_t o[32];
             tmem_ld32(lane_base + col_o + 32 * c, o);
             tmem_wait_ld();
@@ -469,43 +496,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_wait_st();
         }
-        // pass 2: P = exp2(z - max) as bf16 pairs; chunk c's 16 packed
-        // columns land on columns 16c.. of S, which earlier chunks already
-        // read.  The next chunk's load overlaps this chunk's exponentials.
+        // pass 2: P = exp2(z - max) as bf16 pairs; chunk c's 8 packed columns
+        // land on columns 8c.. of this half's S, which earlier chunks already read
         {
-          float ls[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) ls[i] = 0.0f;
-          uint32_t sv[2][32];
-          tmem_ld32(lane_base + col_s, sv[0]);
+          float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          uint32_t sv[2][16];
+          tmem_ld16(lane_base + col_s, sv[0]);
           tmem_wait_ld();
-#pragma unroll 2
-          for (int c = 0; c < 4; ++c) {
-            if (c < 3) tmem_ld32(lane_base + col_s + 32 * (c + 1), sv[(c + 1) & 1]);
-            const uint32_t* v = sv[c & 1];
-            const float bm0 = __shfl_sync(0xffffffffu, c_bias, 2 * c) - m_used;
-            const float bm1 = __shfl_sync(0xffffffffu, c_bias, 2 * c + 1) - m_used;
-            const int n0 = __shfl_sync(0xffffffffu, c_valid, 2 * c), n1 = __shfl_sync(0xffffffffu, c_valid, 2 * c + 1);
-            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int e0 = 2 * i, e1 = e0 + 1;  // column within this 32-column chunk
-              const float bm = i < 8 ? bm0 : bm1;
-              const int nv = i < 8 ? n0 : n1;
-              float x0 = fmaf(__uint_as_float(v[e0]), a.scale_log2, bm);
-              float x1 = fmaf(__uint_as_float(v[e1]), a.scale_log2, bm);
+          for (int c = 0; c < 4; ++c) {
+            if (c < 3) tmem_ld16(lane_base + col_s + 16 * (c + 1), sv[(c + 1) & 1]);
+            const uint32_t* v = sv[c & 1];
+            const float bm = __shfl_sync(0xffffffffu, c_bias, c) - m_used;
+            const int nv = __shfl_sync(0xffffffffu, c_valid, c);
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float x0 = fmaf(__uint_as_float(v[2 * i]), a.scale_log2, bm);
+              float x1 = fmaf(__uint_as_float(v[2 * i + 1]), a.scale_log2, bm);
               if (partial) {
-                x0 = (e0 & 15) < nv ? x0 : -INFINITY;
-                x1 = (e1 & 15) < nv ? x1 : -INFINITY;
+                x0 = 2 * i < nv ? x0 : -INFINITY;
+                x1 = 2 * i + 1 < nv ? x1 : -INFINITY;
               }
               const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-              ls[i & 7] += p0 + p1;
+              ls[i & 3] += p0 + p1;
               pk[i] = pack_bf16x2(p0, p1);
             }
-            tmem_st16(lane_base + col_s + 16 * c, pk);
+            tmem_st8(lane_base + col_s + 8 * c, pk);
             if (c < 3) tmem_wait_ld();
           }
-          l_sum += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+          l_sum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -518,11 +538,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++o_waits;
       tc_fence_after();
-      const float inv = l_sum > 0.0f ? 1.0f / l_sum : 0.0f;
+      float l_tot;
+      if (!exchange(l_sum, false, l_tot)) {
+        ok = false;
+        break;
+      }
+      const float inv = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
       const bool valid = row < w.nrows;
       const int64_t grow = static_cast<int64_t>(w.bh) * a.N + w.row0 + row;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
         tmem_ld32(lane_base + col_o + 32 * c, o);
         tmem_wait_ld();
@@ -531,12 +556,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 16; ++i)
           pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(a.out + grow * D + 32 * c);
+          uint4* dst = reinterpret_cast<uint4*>(a.out + grow * D + (D / 2) * hf + 32 * c);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
-      if (valid && a.lse) a.lse[grow] = (m_used + __log2f(l_sum)) * kLn2;
+      if (valid && hf == 0 && a.lse) a.lse[grow] = (m_used + __log2f(l_tot)) * kLn2;
     }
   }
 
