@@ -299,6 +299,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
       uint32_t ring_pos = 0, q_waits0 = 0, q_waits1 = 0, p_waits0 = 0, p_waits1 = 0;
       uint32_t last_k = 0, last_v = 0;
+      // Shared-memory descriptors are built once: between the k-steps of one
+      // operand only the start-address field (bits 0-13, address >> 4)
+      // changes, and shared addresses stay below 2^18, so a constant add never
+      // carries out of the field.  This keeps the issuing thread's work per
+      // MMA to an add or two.
+      const uint64_t desc_q0 = smem_desc_sw128(base + L::kQOff, 16, 1024);
+      const uint64_t desc_q1 = smem_desc_sw128(base + L::kQOff + L::kQBytes, 16, 1024);
+      const uint64_t desc_k = smem_desc_sw128(base + L::kRingOff, 16, 1024);
+      const uint64_t desc_v = smem_desc_sw128(base + L::kRingOff, L::kChunkBytes, 1024);
       bool ok = true;
       if (a.stall) ok = mbar_wait(bar(L::kBarStall), 0, abort_flag, a.timeout);
       for (int p = blockIdx.x; p < n_pairs && ok; p += gridDim.x) {
@@ -331,15 +340,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             slot = last;
           }
           tc_fence_after();
-          const uint32_t kv = base + L::kRingOff + slot * L::kKVBytes;
+          const uint64_t slot16 = (slot * L::kKVBytes) >> 4;
           if (kind == 0) {
-            const uint32_t q = base + L::kQOff + side * L::kQBytes;
+            const uint64_t da = side ? desc_q1 : desc_q0;
+            const uint64_t db = desc_k + slot16;
             const uint32_t d_s = tmem + (side ? L::kColS1 : L::kColS0);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
-              const uint32_t off = (k >> 2) * L::kChunkBytes + (k & 3) * 32;
-              mma_ss(d_s, smem_desc_sw128(q + off, 16, 1024), smem_desc_sw128(kv + off, 16, 1024), idesc_qk,
-                     k > 0 ? 1u : 0u);
+              const uint64_t off16 = ((k >> 2) * L::kChunkBytes + (k & 3) * 32) >> 4;
+              mma_ss(d_s, da + off16, db + off16, idesc_qk, k > 0 ? 1u : 0u);
             }
             tc_commit(bar(L::kBarSFull + side));
             if (j == T - 1) tc_commit(bar(L::kBarQEmpty + side));
@@ -351,8 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               // keys 0-63: P of the first column half at columns 0-31 of S;
               // keys 64-127: the second half's P at columns 64-95
               const uint32_t pcol = k < 4 ? 8 * k : 64 + 8 * (k - 4);
-              mma_ts(d_o, a_p + pcol, smem_desc_sw128(kv + k * 2048, L::kChunkBytes, 1024), idesc_pv,
-                     (j > 0 || k > 0) ? 1u : 0u);
+              mma_ts(d_o, a_p + pcol, desc_v + slot16 + ((k * 2048) >> 4), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
             }
             if (j == T - 1) tc_commit(bar(L::kBarODone + side));
           }
