@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(L::kBarQFull + i), 1);
       mbar_init(bar(L::kBarQEmpty + i), 1);
       mbar_init(bar(L::kBarSFull + i), 1);
-      mbar_init(bar(L::kBarPFull + i), 256);
+      mbar_init(bar(L::kBarPFull + i), 8);  // one arrival per softmax warp of the tile
       mbar_init(bar(L::kBarODone + i), 1);
     }
     for (int i = 0; i < kRing; ++i) {
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(L::kBarFinal), 1);
     mbar_init(bar(L::kBarStall), 1);  // never arrived at: only the failure-detection hook waits on it
-    for (int i = 0; i < 8; ++i) mbar_init(bar(L::kBarXchg + i), 64);
+    for (int i = 0; i < 8; ++i) mbar_init(bar(L::kBarXchg + i), 2);  // the two warps of a row slice
     *abort_flag = 0;
     *bad_index = 0;
     fence_mbar_init();
@@ -294,7 +294,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // The whole warp runs the loop and waits; one elected lane issues the
+    // MMAs and commits.
+    {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
       uint32_t ring_pos = 0, q_waits0 = 0, q_waits1 = 0, p_waits0 = 0, p_waits1 = 0;
@@ -309,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t desc_k = smem_desc_sw128(base + L::kRingOff, 16, 1024);
       const uint64_t desc_v = smem_desc_sw128(base + L::kRingOff, L::kChunkBytes, 1024);
       bool ok = true;
-      if (a.stall) ok = mbar_wait(bar(L::kBarStall), 0, abort_flag, a.timeout);
+      if (a.stall) ok = mbar_wait_warp(bar(L::kBarStall), 0, abort_flag, a.timeout);
       for (int p = blockIdx.x; p < n_pairs && ok; p += gridDim.x) {
         Work wk[2];
         const bool pr0 = decode_work(a, tph, n_work, 2 * p, wk[0]);
@@ -320,19 +322,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool release = !shared || side == 1;
           if (kind == 0 && j == 0) {
             uint32_t& qw = side ? q_waits1 : q_waits0;
-            if (!mbar_wait(bar(L::kBarQFull + side), qw & 1u, abort_flag, a.timeout)) return false;
+            if (!mbar_wait_warp(bar(L::kBarQFull + side), qw & 1u, abort_flag, a.timeout)) return false;
             ++qw;
           }
           if (kind == 1) {
             uint32_t& pw = side ? p_waits1 : p_waits0;
-            if (!mbar_wait(bar(L::kBarPFull + side), pw & 1u, abort_flag, a.timeout)) return false;
+            if (!mbar_wait_warp(bar(L::kBarPFull + side), pw & 1u, abort_flag, a.timeout)) return false;
             ++pw;
           }
           uint32_t slot;
           uint32_t& last = kind ? last_v : last_k;
           if (acquire) {
             slot = ring_pos % kRing;
-            if (!mbar_wait(bar(L::kBarKVFull + slot), (ring_pos / kRing) & 1u, abort_flag, a.timeout))
+            if (!mbar_wait_warp(bar(L::kBarKVFull + slot), (ring_pos / kRing) & 1u, abort_flag, a.timeout))
               return false;
             ++ring_pos;
             last = slot;
@@ -348,10 +350,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
               const uint64_t off16 = ((k >> 2) * L::kChunkBytes + (k & 3) * 32) >> 4;
-              mma_ss(d_s, da + off16, db + off16, idesc_qk, k > 0 ? 1u : 0u);
+              if (elect_one()) mma_ss(d_s, da + off16, db + off16, idesc_qk, k > 0 ? 1u : 0u);
             }
-            tc_commit(bar(L::kBarSFull + side));
-            if (j == T - 1) tc_commit(bar(L::kBarQEmpty + side));
+            if (elect_one()) {
+              tc_commit(bar(L::kBarSFull + side));
+              if (j == T - 1) tc_commit(bar(L::kBarQEmpty + side));
+            }
           } else {
             const uint32_t a_p = tmem + (side ? L::kColS1 : L::kColS0);
             const uint32_t d_o = tmem + (side ? L::kColO1 : L::kColO0);
@@ -360,16 +364,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               // keys 0-63: P of the first column half at columns 0-31 of S;
               // keys 64-127: the second half's P at columns 64-95
               const uint32_t pcol = k < 4 ? 8 * k : 64 + 8 * (k - 4);
-              mma_ts(d_o, a_p + pcol, desc_v + slot16 + ((k * 2048) >> 4), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+              if (elect_one())
+                mma_ts(d_o, a_p + pcol, desc_v + slot16 + ((k * 2048) >> 4), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
             }
-            if (j == T - 1) tc_commit(bar(L::kBarODone + side));
+            if (j == T - 1 && elect_one()) tc_commit(bar(L::kBarODone + side));
           }
-          if (release) tc_commit(bar(L::kBarKVEmpty + slot));
+          if (release && elect_one()) tc_commit(bar(L::kBarKVEmpty + slot));
           return true;
         });
       }
       // every MMA must be complete before tensor memory is freed
-      tc_commit(bar(L::kBarFinal));
+      if (elect_one()) tc_commit(bar(L::kBarFinal));
+      __syncwarp();
       drain_wait(bar(L::kBarFinal), 0);
     }
   } else if (warp < 16) {
@@ -395,8 +401,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto exchange = [&](float v, bool is_max, float& out) -> bool {
       float* xchg = is_max ? xchg_max : xchg_sum;
       xchg[hf * 128 + row] = v;
-      mbar_arrive(xbar);
-      if (!mbar_wait(xbar, x_waits & 1u, abort_flag, a.timeout)) return false;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xbar);
+      if (!mbar_wait_warp(xbar, x_waits & 1u, abort_flag, a.timeout)) return false;
       ++x_waits;
       const float o = xchg[(1 - hf) * 128 + row];
       out = is_max ? fmaxf(v, o) : v + o;
@@ -445,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float c_bias;
         int c_valid;
         decode(j, cur_idx, cur_lw, c_bias, c_valid);
-        if (!mbar_wait(bar(L::kBarSFull + x), s_waits & 1u, abort_flag, a.timeout)) {
+        if (!mbar_wait_warp(bar(L::kBarSFull + x), s_waits & 1u, abort_flag, a.timeout)) {
           ok = false;
           break;
         }
@@ -537,10 +544,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(L::kBarPFull + x));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::kBarPFull + x));
       }
       if (!ok) break;
-      if (!mbar_wait(bar(L::kBarODone + x), o_waits & 1u, abort_flag, a.timeout)) {
+      if (!mbar_wait_warp(bar(L::kBarODone + x), o_waits & 1u, abort_flag, a.timeout)) {
         ok = false;
         break;
       }
