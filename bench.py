@@ -38,6 +38,25 @@ if ROOT not in sys.path:
 METRIC = "sparse IS-attention ms/call + computed TFLOP/s vs B200 BF16 peak, per shape"
 UNIT = "TFLOP/s (computed)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
+# launch, per head, from an ncu capture of the wan14_10 layer cut to 4 heads.
+# Q, K, V and O all scale with the head count.  The figure holds only for the
+# kernel source whose SHA-256 starts with the recorded prefix; for any other
+# source (or workload) the roofline reports traffic as null.
+ATTN_TRAFFIC = {"workload": "wan14_10", "src_sha256_prefix": "cc314330dacf6be6", "bytes_per_head": 308.0e6 / 4}
+
+
+def attn_traffic(workload, heads):
+    import hashlib
+    src = os.path.join(ROOT, "block_sparse_importance_b200", "csrc", "attn.cu")
+    try:
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    if workload != ATTN_TRAFFIC["workload"] or not sha.startswith(ATTN_TRAFFIC["src_sha256_prefix"]):
+        return None
+    return ATTN_TRAFFIC["bytes_per_head"] * heads
 
 
 def load_peaks():
@@ -239,7 +258,11 @@ def main():
     aws = torch.empty(aws_n + 256, dtype=torch.uint8, device=dev) if aws_n else None
 
     def step(ev=None):
+        if ev is not None:
+            ev[2].record(stream)
         isa.score(q, k, lay, w.n_clusters, w.n_iters, mass=mass, workspace=sws, ctx=ctx)
+        if ev is not None:
+            ev[3].record(stream)
         isa.select(mass, lay, w.n_exact, w.n_sample, w.seed, idx=idx, log_w=lw, ctx=ctx)
         if ev is not None:
             ev[0].record(stream)
@@ -254,8 +277,7 @@ def main():
         raise RuntimeError("device status after warm-up: %s" % isa.status_string(st))
     flops = plan_flops(idx.cpu().numpy(), inp.offsets, N, w.k_block, d)   # per step (per rank)
 
-    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
+    attn_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(gpu_query_id(dev)) as clk:
         if world > 1:
@@ -273,11 +295,13 @@ def main():
     if st != isa.ISA_OK:
         raise RuntimeError("device status after timing: %s" % isa.status_string(st))
     elapsed_ms = t0.elapsed_time(t1)
-    attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / args.steps
+    attn_ms = sum(e[0].elapsed_time(e[1]) for e in attn_ev) / args.steps
+    score_ms = sum(e[2].elapsed_time(e[3]) for e in attn_ev) / args.steps
+    select_ms = sum(e[3].elapsed_time(e[0]) for e in attn_ev) / args.steps
     if world > 1:
-        tt = torch.tensor([elapsed_ms, attn_ms], device=dev)
+        tt = torch.tensor([elapsed_ms, attn_ms, score_ms, select_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms, attn_ms = float(tt[0]), float(tt[1])
+        elapsed_ms, attn_ms, score_ms, select_ms = (float(x) for x in tt)
     ms_step = elapsed_ms / args.steps
     value = world * flops / (ms_step * 1e-3) / 1e12
 
@@ -285,8 +309,20 @@ def main():
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     achieved = flops / (attn_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "kernel": "attn_kernel<128>",
+                "frac": achieved / peak, "traffic": attn_traffic(args.workload, H * B),
+                "traffic_unit": "bytes per launch", "kernel": "attn_kernel<128>",
                 "peak_source": "%s bf16_tflops_sustained (kernel timed inside a multi-kernel step loop)" % peak_src}
+
+    # the two HBM-bound stages: algorithmic bytes over their event-timed durations
+    hbm = float(peaks.get("hbm_gbs"))
+    score_bytes = 2 * B * H * N * d * 2 + 4 * B * H * G * nK     # Q and K read, mass written
+    select_bytes = B * H * G * (4 * nK + 8 * S)                   # mass read, plan written
+    stages = {
+        "score": {"ms": score_ms, "bytes": score_bytes, "gbs": score_bytes / (score_ms * 1e-3) / 1e9},
+        "select": {"ms": select_ms, "bytes": select_bytes, "gbs": select_bytes / (select_ms * 1e-3) / 1e9},
+    }
+    for v_ in stages.values():
+        v_["frac_hbm"] = v_["gbs"] / hbm
 
     # dense limit, same tensors (context for the speedup analogue)
     dense_ms = None
@@ -346,7 +382,7 @@ def main():
                 "dense_attention_ms": dense_ms,
                 "sparse_vs_dense": (dense_ms / attn_ms) if dense_ms else None,
                 "computed_tflop_per_step": flops / 1e12,
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
         print(json.dumps(line), flush=True)
     if world > 1:
