@@ -60,6 +60,7 @@ struct __align__(16) TileDesc {
 
 struct AttnArgs {
   int BH, N, G, S, Bk, nK, q_block, mode;
+  int bk_shift;  // log2(Bk): plan positions are split into block and offset by shifts
   int tiles_per_head;  // groups / dense modes
   int T;               // KV tiles per query tile
   const int32_t* idx;
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_pairs = (n_work + 1) >> 1;
   const int T = a.T;
   const bool dense = a.mode == kAttnDense;
-  const int bpt = dense ? 1 : kTileRows / a.Bk;  // plan blocks per KV tile
+  const int bpt = dense ? 1 : kTileRows >> a.bk_shift;  // plan blocks per KV tile
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         rb = -1;
         rlw = 0.0f;
         if (!dense && lane < 4) {
-          const int s = (jj * kTileRows + 64 * hf + lane * 16) / a.Bk;
+          const int s = (jj * kTileRows + 64 * hf + lane * 16) >> a.bk_shift;
           if (s < a.S) {
             rb = a.idx[prow + s];
             rlw = a.log_w[prow + s];
@@ -436,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (dense) {
             valid_o = max(0, min(16, a.N - pos));
           } else if (rb >= 0 && rb < a.nK) {
-            const int within = pos - (pos / a.Bk) * a.Bk;
+            const int within = pos & (a.Bk - 1);
             valid_o = max(0, min(16, min(a.Bk, a.N - rb * a.Bk) - within));
             bias_o = rlw * kLog2e;
           }
@@ -651,6 +652,8 @@ int launch_d(const AttnLaunch& l, const void* q, const void* k, const void* v, c
   a.G = l.G;
   a.S = l.S;
   a.Bk = l.Bk;
+  a.bk_shift = 0;
+  while ((1 << a.bk_shift) < l.Bk) ++a.bk_shift;
   a.nK = (l.N + l.Bk - 1) / l.Bk;
   a.q_block = l.q_block;
   a.mode = l.mode;
