@@ -123,10 +123,16 @@ __global__ void __launch_bounds__(kScoreThreads) kmeans_kernel(const uint16_t* _
   }
   const int n = r1 - r0;
   const uint16_t* qg = q + (bh * N + r0) * D;
-  for (int i = tid; i < 16 * D; i += kScoreThreads) {
+  // initial centroids: rows floor(c n / C), worked out once per centroid;
+  // the trip count is fixed so that all of a thread's gathers are in flight
+  // together
+  if (tid < 16) assign[tid] = static_cast<int>((static_cast<int64_t>(tid) * n) / max(C, 1));
+  __syncthreads();
+#pragma unroll
+  for (int k2 = 0; k2 < 16 * D / kScoreThreads; ++k2) {
+    const int i = tid + k2 * kScoreThreads;
     const int c = i / D, j = i - c * D;
-    const int r = static_cast<int>((static_cast<int64_t>(c) * n) / C);
-    mu[i] = (c < C && n > 0) ? bf16_to_f(qg[static_cast<int64_t>(r) * D + j]) : 0.0f;
+    mu[i] = (c < C && n > 0) ? bf16_to_f(qg[static_cast<int64_t>(assign[c]) * D + j]) : 0.0f;
   }
   const bool one_chunk = n <= kChunkRows;
   const uint32_t xs_base = smem_addr(xs), mhi_base = smem_addr(mhi), mlo_base = smem_addr(mlo);
@@ -138,8 +144,9 @@ __global__ void __launch_bounds__(kScoreThreads) kmeans_kernel(const uint16_t* _
   const int t_row = (lane & 7) + ((lane >> 3) & 1) * 8, t_col = (lane >> 4) * 8;
   __syncthreads();
   for (int it = 0; it < iters; ++it) {
-    // split the centroids into bf16 hi + lo and take |mu|^2
-    for (int i = tid; i < 16 * D; i += kScoreThreads) {
+    // split the centroids into bf16 hi + lo and take |mu|^2 (rows c >= C
+    // stay zero from the first round: their mu is zero)
+    for (int i = tid; i < (it == 0 ? 16 : C) * D; i += kScoreThreads) {
       const int c = i / D, j = i - c * D;
       const float m = mu[i];
       const uint16_t hi = bf16_bits_rn(m);
@@ -147,7 +154,7 @@ __global__ void __launch_bounds__(kScoreThreads) kmeans_kernel(const uint16_t* _
       mhi[c * XS + j] = hi;
       mlo[c * XS + j] = lo;
     }
-    for (int c = warp; c < 16; c += kScoreThreads / 32) {
+    for (int c = warp; c < C; c += kScoreThreads / 32) {
       float acc = 0.0f;
       for (int j = lane; j < D; j += 32) acc = fmaf(mu[c * D + j], mu[c * D + j], acc);
 #pragma unroll
@@ -164,13 +171,17 @@ __global__ void __launch_bounds__(kScoreThreads) kmeans_kernel(const uint16_t* _
     for (int cs = 0; cs < n; cs += kChunkRows) {
       const int rc = min(kChunkRows, n - cs);
       if (!(one_chunk && it > 0)) {
-        // rows [cs, cs+rc) into the padded buffer; rows past rc are zeroed
-        for (int i = tid; i < kChunkRows * (D / 8); i += kScoreThreads) {
+        // rows [cs, cs+rc) into the padded buffer by asynchronous 16-byte
+        // copies, all in flight together; rows past rc are zero-filled
+#pragma unroll
+        for (int k2 = 0; k2 < kChunkRows * (D / 8) / kScoreThreads; ++k2) {
+          const int i = tid + k2 * kScoreThreads;
           const int r = i / (D / 8), c16 = i - r * (D / 8);
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (r < rc) v = reinterpret_cast<const uint4*>(qg + static_cast<int64_t>(cs + r) * D)[c16];
-          *reinterpret_cast<uint4*>(xs + r * XS + c16 * 8) = v;
+          const bool in = r < rc;
+          const uint16_t* src = in ? qg + static_cast<int64_t>(cs + r) * D + c16 * 8 : qg;
+          cp_async16_zfill(xs_base + 2u * (r * XS + c16 * 8), src, in ? 16u : 0u);
         }
+        cp_async_wait_all();
         __syncthreads();
       }
       // ---- assignment: warp w takes rows 16w .. 16w+15
@@ -257,14 +268,20 @@ __global__ void __launch_bounds__(kScoreThreads) kmeans_kernel(const uint16_t* _
     }
     // ---- update: each (cluster, column) is owned by one thread
 #pragma unroll
-    for (int nt = 0; nt < NTD; ++nt)
+    for (int h = 0; h < 2; ++h) {
+      const int c = gq + 8 * h;
+      const int nc = cnt[c];
+      if (c < C && nc > 0) {
+        const float nf = static_cast<float>(nc);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = gq + 8 * (e >> 1);
-        const int j = 8 * (NTD * warp + nt) + 2 * tq + (e & 1);
-        const int nc = cnt[c];
-        if (c < C && nc > 0) mu[c * D + j] = sums[nt][e] / static_cast<float>(nc);
+        for (int nt = 0; nt < NTD; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = 8 * (NTD * warp + nt) + 2 * tq + e;
+            mu[c * D + j] = __fdiv_rn(sums[nt][2 * h + e], nf);
+          }
       }
+    }
     __syncthreads();
   }
   const int64_t t = bh * G + g;
