@@ -9,11 +9,11 @@
 // Three kernels:
 //   key_means_kernel  kbar_b = mean of the valid rows of key block b, stored
 //                     as a bf16 hi + lo pair;
-//   kmeans_kernel     per (batch*head, group): Lloyd's k-means, centroids
-//                     initialised at rows floor(c n / C), `iters` rounds of
-//                     nearest-centroid assignment (squared distance, ties to
-//                     the lower c) and mean update; rows stream through
-//                     shared memory 128 at a time;
+//   kmeans_warp_kernel  per (batch*head, group), one warp: Lloyd's
+//                     k-means, centroids initialised at rows floor(c n / C),
+//                     `iters` rounds of nearest-centroid assignment (squared
+//                     distance, ties to the lower c) and mean update; rows
+//                     stream through shared memory 128 at a time;
 //   mass_kernel       per (batch*head, 128 / C' groups): logits
 //                     l = scale mu_c . kbar_b + ln L_b, a first pass for the
 //                     per-centroid softmax max and sum over all key blocks, a
@@ -83,217 +83,258 @@ __global__ void __launch_bounds__(kScoreThreads) key_means_kernel(const uint16_t
 // One CTA (8 warps) per (batch*head, group).  Rows stream through shared
 // memory 128 at a time (a group of <= 128 rows is loaded once), rows padded to
 // D + 8 elements so that ldmatrix reads are free of bank conflicts.
+// ---------------------------------------------- k-means, one warp per group
 // Assignment: dist_c = |mu_c|^2 - 2 x.mu_c (|x|^2 is common to all c) with the
 // dots on tensor cores: x is exact in bf16 and mu_c is split into bf16
 // hi + lo parts (relative error 2^-18), two mma.sync per 16x8x16 tile.
 // Update: the cluster sums are a one-hot product (assignment^T x) on tensor
 // cores, exact products accumulated in fp32; mu_c = sum_c / n_c.
-template <int D, int NTC>
-__global__ void __launch_bounds__(kScoreThreads) kmeans_kernel(const uint16_t* __restrict__ q, int N, int G,
-                                                               int q_block, const int32_t* __restrict__ off, int C,
-                                                               int iters, float* __restrict__ centroids,
-                                                               int32_t* __restrict__ counts, int* status) {
-  using namespace isa_dev;
-  constexpr int XS = D + 8;            // padded row stride (elements)
-  constexpr int KSTEPS = D / 16;       // k-steps of the dot products
-  constexpr int NTD = D / 64;          // 8-column n-tiles of the sums per warp
-  extern __shared__ __align__(16) uint8_t sm[];
-  uint16_t* xs = reinterpret_cast<uint16_t*>(sm);                          // [128][XS]
-  uint16_t* mhi = xs + kChunkRows * XS;                                     // [16][XS]
-  uint16_t* mlo = mhi + 16 * XS;                                            // [16][XS]
-  float* mu = reinterpret_cast<float*>(mlo + 16 * XS);                      // [16][D]
-  float* musq = mu + 16 * D;                                                // [16]
-  int* cnt = reinterpret_cast<int*>(musq + 16);                             // [16]
-  int* assign = cnt + 16;                                                   // [128]
-  const int g = blockIdx.x;
-  const int64_t bh = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gq = lane >> 2, tq = lane & 3;
-  int r0, r1;
-  if (off) {
-    r0 = off[g];
-    r1 = off[g + 1];
-    if (r0 < 0 || r1 > N || r1 <= r0) {  // malformed offsets: leave an empty group
-      if (tid == 0) atomicCAS(status, 0, kStatusDeviceCheck);
-      r1 = r0 = 0;
-    }
-  } else {
-    r0 = g * q_block;
-    r1 = min(N, r0 + q_block);
-  }
-  const int n = r1 - r0;
-  const uint16_t* qg = q + (bh * N + r0) * D;
-  // initial centroids: rows floor(c n / C), worked out once per centroid;
-  // the trip count is fixed so that all of a thread's gathers are in flight
-  // together
-  if (tid < 16) assign[tid] = static_cast<int>((static_cast<int64_t>(tid) * n) / max(C, 1));
-  __syncthreads();
-#pragma unroll
-  for (int k2 = 0; k2 < 16 * D / kScoreThreads; ++k2) {
-    const int i = tid + k2 * kScoreThreads;
-    const int c = i / D, j = i - c * D;
-    mu[i] = (c < C && n > 0) ? bf16_to_f(qg[static_cast<int64_t>(assign[c]) * D + j]) : 0.0f;
-  }
-  const bool one_chunk = n <= kChunkRows;
-  const uint32_t xs_base = smem_addr(xs), mhi_base = smem_addr(mhi), mlo_base = smem_addr(mlo);
-  // ldmatrix row address of this lane for a 16x16 A tile at (row0, col0)
-  const int a_row = (lane & 7) + ((lane >> 3) & 1) * 8, a_col = (lane >> 4) * 8;
-  // x2 B tile (8 centroid rows x 16 k): lanes 0-7 k 0-7, lanes 8-15 k 8-15
-  const int b_row = lane & 7, b_col = ((lane >> 3) & 1) * 8;
-  // x4 / x2 trans B tile from x rows: matrices (k 0-7, n 0-7), (k 8-15, n 0-7), (k 0-7, n 8-15), (k 8-15, n 8-15)
-  const int t_row = (lane & 7) + ((lane >> 3) & 1) * 8, t_col = (lane >> 4) * 8;
-  __syncthreads();
-  for (int it = 0; it < iters; ++it) {
-    // split the centroids into bf16 hi + lo and take |mu|^2 (rows c >= C
-    // stay zero from the first round: their mu is zero)
-    for (int i = tid; i < (it == 0 ? 16 : C) * D; i += kScoreThreads) {
-      const int c = i / D, j = i - c * D;
-      const float m = mu[i];
-      const uint16_t hi = bf16_bits_rn(m);
-      const uint16_t lo = bf16_bits_rn(m - bf16_bits_to_f(hi));
-      mhi[c * XS + j] = hi;
-      mlo[c * XS + j] = lo;
-    }
-    for (int c = warp; c < C; c += kScoreThreads / 32) {
-      float acc = 0.0f;
-      for (int j = lane; j < D; j += 32) acc = fmaf(mu[c * D + j], mu[c * D + j], acc);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) musq[c] = acc;
-    }
-    if (tid < 16) cnt[tid] = 0;
-    float sums[NTD][4];
-#pragma unroll
-    for (int i = 0; i < NTD; ++i)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) sums[i][k] = 0.0f;
-    __syncthreads();
-    for (int cs = 0; cs < n; cs += kChunkRows) {
-      const int rc = min(kChunkRows, n - cs);
-      if (!(one_chunk && it > 0)) {
-        // rows [cs, cs+rc) into the padded buffer by asynchronous 16-byte
-        // copies, all in flight together; rows past rc are zero-filled
-#pragma unroll
-        for (int k2 = 0; k2 < kChunkRows * (D / 8) / kScoreThreads; ++k2) {
-          const int i = tid + k2 * kScoreThreads;
-          const int r = i / (D / 8), c16 = i - r * (D / 8);
-          const bool in = r < rc;
-          const uint16_t* src = in ? qg + static_cast<int64_t>(cs + r) * D + c16 * 8 : qg;
-          cp_async16_zfill(xs_base + 2u * (r * XS + c16 * 8), src, in ? 16u : 0u);
-        }
-        cp_async_wait_all();
-        __syncthreads();
-      }
-      // ---- assignment: warp w takes rows 16w .. 16w+15
-      if (16 * warp < rc) {
-        float acc[NTC][4];
-#pragma unroll
-        for (int i = 0; i < NTC; ++i)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc[i][k] = 0.0f;
-#pragma unroll
-        for (int ks = 0; ks < KSTEPS; ++ks) {
-          uint32_t a[4];
-          ldsm_x4(a, xs_base + 2u * ((16 * warp + a_row) * XS + ks * 16 + a_col));
-#pragma unroll
-          for (int nt = 0; nt < NTC; ++nt) {
-            uint32_t bh2[2], bl2[2];
-            const uint32_t off_b = 2u * ((8 * nt + b_row) * XS + ks * 16 + b_col);
-            ldsm_x2(bh2, mhi_base + off_b);
-            ldsm_x2(bl2, mlo_base + off_b);
-            mma_16816(acc[nt], a, bh2[0], bh2[1]);
-            mma_16816(acc[nt], a, bl2[0], bl2[1]);
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {  // rows gq and gq + 8
-          float best = INFINITY;
-          int bi = 0;
-#pragma unroll
-          for (int nt = 0; nt < NTC; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int c = 8 * nt + 2 * tq + e;
-              const float dist = musq[c] - 2.0f * acc[nt][2 * h + e];
-              if (c < C && dist < best) {
-                best = dist;
-                bi = c;
-              }
-            }
-#pragma unroll
-          for (int o = 1; o <= 2; o <<= 1) {
-            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ob < best || (ob == best && oi < bi)) {
-              best = ob;
-              bi = oi;
-            }
-          }
-          const int r = 16 * warp + gq + 8 * h;
-          if (tq == 0) {
-            if (r < rc) {
-              assign[r] = bi;
-              atomicAdd(&cnt[bi], 1);
-            } else {
-              assign[r] = -1;
-            }
-          }
-        }
-      } else if (lane < 16) {
-        assign[16 * warp + lane] = -1;
-      }
-      __syncthreads();
-      // ---- cluster sums: one-hot(assign)^T x; warp w owns columns [8 NTD w, 8 NTD (w+1))
-      for (int k0 = 0; k0 < rc; k0 += 16) {
-        uint32_t a[4];
-        const int ka = k0 + 2 * tq, kb = ka + 8;
-        const int s0 = assign[ka], s1 = assign[ka + 1], s2 = assign[kb], s3 = assign[kb + 1];
-        const uint32_t one = 0x3F80u;
-        a[0] = (s0 == gq ? one : 0u) | ((s1 == gq ? one : 0u) << 16);
-        a[1] = (s0 == gq + 8 ? one : 0u) | ((s1 == gq + 8 ? one : 0u) << 16);
-        a[2] = (s2 == gq ? one : 0u) | ((s3 == gq ? one : 0u) << 16);
-        a[3] = (s2 == gq + 8 ? one : 0u) | ((s3 == gq + 8 ? one : 0u) << 16);
-        if constexpr (NTD == 2) {
-          uint32_t b[4];
-          ldsm_x4_trans(b, xs_base + 2u * ((k0 + t_row) * XS + 16 * warp + t_col));
-          mma_16816(sums[0], a, b[0], b[1]);
-          mma_16816(sums[1], a, b[2], b[3]);
-        } else {
-          uint32_t b[2];
-          ldsm_x2_trans(b, xs_base + 2u * ((k0 + (lane & 15)) * XS + 8 * warp));
-          mma_16816(sums[0], a, b[0], b[1]);
-        }
-      }
-      __syncthreads();
-    }
-    // ---- update: each (cluster, column) is owned by one thread
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = gq + 8 * h;
-      const int nc = cnt[c];
-      if (c < C && nc > 0) {
-        const float nf = static_cast<float>(nc);
-#pragma unroll
-        for (int nt = 0; nt < NTD; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int j = 8 * (NTD * warp + nt) + 2 * tq + e;
-            mu[c * D + j] = __fdiv_rn(sums[nt][2 * h + e], nf);
-          }
-      }
-    }
-    __syncthreads();
-  }
-  const int64_t t = bh * G + g;
-  for (int i = tid; i < C * D; i += kScoreThreads) centroids[t * C * D + i] = mu[i];
-  if (tid < C) counts[t * C + tid] = cnt[tid];
-}
+// Every step of a group runs in one warp, with no block-wide barriers:
+//   * the lane holding row gq of an mma.sync C tile also holds, in the B
+//     fragment layout, dimensions 16 ks + 2 tq + {0, 1, 8, 9} of centroid
+//     gq (and gq + 8): the cluster sums come out of the one-hot product in
+//     exactly the registers the next round's distance products read, so the
+//     centroids never leave registers;
+//   * the count of each cluster is the sum over an extra column of ones
+//     stored beside every valid row (a row past the group's end holds 0);
+//   * rows stream through the warp's shared-memory buffer 128 at a time by
+//     cp.async.
+constexpr int kKmWarps = 6;
 
 template <int D>
-size_t kmeans_smem_bytes() {
-  constexpr int XS = D + 8;
-  return (kChunkRows * XS + 2 * 16 * XS) * 2 + (16 * D + 16) * 4 + (16 + kChunkRows) * 4;
+struct KmLayout {
+  static constexpr int XS = D + 8;  // padded row (elements); column D holds 1.0 for a valid row
+  static constexpr uint32_t kXBytes = kChunkRows * XS * 2;
+  static constexpr uint32_t kWarpBytes = kXBytes + kChunkRows * 4;  // + the chunk's assignments
+  static constexpr uint32_t kAlloc = kKmWarps * kWarpBytes;
+};
+
+template <int D, int NTC>
+__global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16_t* __restrict__ q, int BH, int N,
+                                                                    int G, int q_block,
+                                                                    const int32_t* __restrict__ off, int C,
+                                                                    int iters, float* __restrict__ centroids,
+                                                                    int32_t* __restrict__ counts, int* status) {
+  using namespace isa_dev;
+  using L = KmLayout<D>;
+  constexpr int XS = L::XS;
+  constexpr int KSTEPS = D / 16;  // k-steps of the distance products
+  constexpr int NTS = D / 8 + 1;  // n-tiles of the cluster sums; the last one holds the counts
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(sm + warp * L::kWarpBytes);
+  int* assign = reinterpret_cast<int*>(sm + warp * L::kWarpBytes + L::kXBytes);
+  const uint32_t xs_base = smem_addr(xs);
+  // ldmatrix row address of this lane: x4 A tile at (row0, col0); x4 trans B
+  // tile from x rows: matrices (k 0-7, n 0-7), (k 8-15, n 0-7), (k 0-7, n 8-15), (k 8-15, n 8-15)
+  const int a_row = (lane & 7) + ((lane >> 3) & 1) * 8, a_col = (lane >> 4) * 8;
+  const int t_row = (lane & 7) + ((lane >> 3) & 1) * 8, t_col = (lane >> 4) * 8;
+  const int64_t n_items = static_cast<int64_t>(BH) * G;
+  for (int64_t item = static_cast<int64_t>(blockIdx.x) * kKmWarps + warp; item < n_items;
+       item += static_cast<int64_t>(gridDim.x) * kKmWarps) {
+    const int64_t bh = item / G;
+    const int g = static_cast<int>(item - bh * G);
+    int r0, r1;
+    if (off) {
+      r0 = off[g];
+      r1 = off[g + 1];
+      if (r0 < 0 || r1 > N || r1 <= r0) {  // malformed offsets: leave an empty group
+        if (lane == 0) atomicCAS(status, 0, kStatusDeviceCheck);
+        r1 = r0 = 0;
+      }
+    } else {
+      r0 = g * q_block;
+      r1 = min(N, r0 + q_block);
+    }
+    const int n = r1 - r0;
+    const uint16_t* qg = q + (bh * N + r0) * D;
+    // this lane's dimensions of centroids gq (+ 8), initialised at rows
+    // floor(c n / C); all gathers of a lane are in flight together
+    float mu[NTC][KSTEPS][4];
+#pragma unroll
+    for (int h = 0; h < NTC; ++h) {
+      const int c = gq + 8 * h;
+      const int r = (c < C && n > 0) ? static_cast<int>((static_cast<int64_t>(c) * n) / C) : -1;
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ++ks)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int dim = 16 * ks + 2 * tq + (e & 1) + 8 * (e >> 1);
+          mu[h][ks][e] = r >= 0 ? bf16_to_f(qg[static_cast<int64_t>(r) * D + dim]) : 0.0f;
+        }
+    }
+    int cnt[NTC];
+#pragma unroll
+    for (int h = 0; h < NTC; ++h) cnt[h] = 0;
+    const bool one_chunk = n <= kChunkRows;
+    for (int it = 0; it < iters; ++it) {
+      // centroids as bf16 hi + lo B fragments, and |mu_c|^2
+      uint32_t bhi[NTC][KSTEPS][2], blo[NTC][KSTEPS][2];
+      float nsq[NTC];
+#pragma unroll
+      for (int h = 0; h < NTC; ++h) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks)
+#pragma unroll
+          for (int p = 0; p < 2; ++p) {
+            const float x0 = mu[h][ks][2 * p], x1 = mu[h][ks][2 * p + 1];
+            const uint32_t hi = pack_bf16x2(x0, x1);
+            const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);
+            bhi[h][ks][p] = hi;
+            blo[h][ks][p] = pack_bf16x2(x0 - h0, x1 - h1);
+            acc = fmaf(x0, x0, acc);
+            acc = fmaf(x1, x1, acc);
+          }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        nsq[h] = acc;
+      }
+      // |mu|^2 of the two centroids (columns 2 tq, 2 tq + 1) of each n-tile
+      float msq[NTC][2];
+#pragma unroll
+      for (int nt = 0; nt < NTC; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) msq[nt][e] = __shfl_sync(0xffffffffu, nsq[nt], 4 * (2 * tq + e));
+      float sums[NTS][4];
+#pragma unroll
+      for (int i = 0; i < NTS; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sums[i][k] = 0.0f;
+      for (int cs = 0; cs < n; cs += kChunkRows) {
+        const int rc = min(kChunkRows, n - cs);
+        if (!(one_chunk && it > 0)) {
+          __syncwarp();  // every lane is done with the previous rows
+#pragma unroll 8
+          for (int k2 = 0; k2 < kChunkRows * (D / 8) / 32; ++k2) {
+            const int i = lane + 32 * k2;
+            const int r = i / (D / 8), c16 = i - r * (D / 8);
+            const bool in = r < rc;
+            const uint16_t* src = in ? qg + static_cast<int64_t>(cs + r) * D + c16 * 8 : qg;
+            cp_async16_zfill(xs_base + 2u * (r * XS + c16 * 8), src, in ? 16u : 0u);
+          }
+          for (int r = lane; r < kChunkRows; r += 32)
+            *reinterpret_cast<uint4*>(xs + r * XS + D) = make_uint4(r < rc ? 0x3F80u : 0u, 0u, 0u, 0u);
+          cp_async_wait_all();
+          __syncwarp();
+        }
+        // assignment: dist_c = |mu_c|^2 - 2 x.mu_c; argmin over c (ties to the
+        // lower c) of rows gq and gq + 8 of row tile rt
+        auto pick = [&](int rt, const float (&acc)[NTC][4]) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            float best = INFINITY;
+            int bi = 0;
+#pragma unroll
+            for (int nt = 0; nt < NTC; ++nt)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int c = 8 * nt + 2 * tq + e;
+                const float dist = msq[nt][e] - 2.0f * acc[nt][2 * hh + e];
+                if (c < C && dist < best) {
+                  best = dist;
+                  bi = c;
+                }
+              }
+#pragma unroll
+            for (int o = 1; o <= 2; o <<= 1) {
+              const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+              const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+              if (ob < best || (ob == best && oi < bi)) {
+                best = ob;
+                bi = oi;
+              }
+            }
+            const int r = 16 * rt + gq + 8 * hh;
+            if (tq == 0) assign[r] = r < rc ? bi : -1;
+          }
+        };
+        const int nrt = (rc + 15) / 16;  // row tiles holding rows of the group
+        {
+          for (int rt = 0; rt < kChunkRows / 16; ++rt) {
+            if (rt >= nrt) {
+              if (lane < 16) assign[16 * rt + lane] = -1;
+              continue;
+            }
+            float acc[NTC][4];
+#pragma unroll
+            for (int i = 0; i < NTC; ++i)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) acc[i][k] = 0.0f;
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS; ++ks) {
+              uint32_t a[4];
+              ldsm_x4(a, xs_base + 2u * ((16 * rt + a_row) * XS + ks * 16 + a_col));
+#pragma unroll
+              for (int nt = 0; nt < NTC; ++nt) {
+                mma_16816(acc[nt], a, bhi[nt][ks][0], bhi[nt][ks][1]);
+                mma_16816(acc[nt], a, blo[nt][ks][0], blo[nt][ks][1]);
+              }
+            }
+            pick(rt, acc);
+          }
+        }
+        __syncwarp();
+        // cluster sums (and counts, from the column of ones): one-hot^T x
+        for (int k0 = 0; k0 < rc; k0 += 16) {
+          uint32_t a[4];
+          const int ka = k0 + 2 * tq, kb = ka + 8;
+          const int s0 = assign[ka], s1 = assign[ka + 1], s2 = assign[kb], s3 = assign[kb + 1];
+          const uint32_t one = 0x3F80u;
+          a[0] = (s0 == gq ? one : 0u) | ((s1 == gq ? one : 0u) << 16);
+          a[1] = (s0 == gq + 8 ? one : 0u) | ((s1 == gq + 8 ? one : 0u) << 16);
+          a[2] = (s2 == gq ? one : 0u) | ((s3 == gq ? one : 0u) << 16);
+          a[3] = (s2 == gq + 8 ? one : 0u) | ((s3 == gq + 8 ? one : 0u) << 16);
+#pragma unroll
+          for (int p = 0; p < D / 16; ++p) {
+            uint32_t b[4];
+            ldsm_x4_trans(b, xs_base + 2u * ((k0 + t_row) * XS + 16 * p + t_col));
+            mma_16816(sums[2 * p], a, b[0], b[1]);
+            mma_16816(sums[2 * p + 1], a, b[2], b[3]);
+          }
+          uint32_t b2[2];
+          ldsm_x2_trans(b2, xs_base + 2u * ((k0 + (lane & 15)) * XS + D));
+          mma_16816(sums[D / 8], a, b2[0], b2[1]);
+        }
+      }
+      // counts: column 0 of the last n-tile, held by the quad's first lane
+#pragma unroll
+      for (int h = 0; h < NTC; ++h)
+        cnt[h] = static_cast<int>(__shfl_sync(0xffffffffu, sums[D / 8][2 * h], lane & ~3));
+      // update: mu_c = sum_c / n_c in the registers the next round reads
+#pragma unroll
+      for (int h = 0; h < NTC; ++h) {
+        const int c = gq + 8 * h;
+        if (c < C && cnt[h] > 0) {
+          const float inv = 1.0f / static_cast<float>(cnt[h]);
+#pragma unroll
+          for (int ks = 0; ks < KSTEPS; ++ks) {
+            mu[h][ks][0] = sums[2 * ks][2 * h] * inv;
+            mu[h][ks][1] = sums[2 * ks][2 * h + 1] * inv;
+            mu[h][ks][2] = sums[2 * ks + 1][2 * h] * inv;
+            mu[h][ks][3] = sums[2 * ks + 1][2 * h + 1] * inv;
+          }
+        }
+      }
+    }
+    const int64_t t = bh * G + g;
+#pragma unroll
+    for (int h = 0; h < NTC; ++h) {
+      const int c = gq + 8 * h;
+      if (c < C) {
+        float* dst = centroids + (t * C + c) * D;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          *reinterpret_cast<float2*>(dst + 16 * ks + 2 * tq) = make_float2(mu[h][ks][0], mu[h][ks][1]);
+          *reinterpret_cast<float2*>(dst + 16 * ks + 8 + 2 * tq) = make_float2(mu[h][ks][2], mu[h][ks][3]);
+        }
+        if (tq == 0) counts[t * C + c] = cnt[h];
+      }
+    }
+  }
 }
+
 
 // ------------------------------------------------------------------ mass
 // One CTA per (batch*head, 128 centroid rows = 128 / Cp groups; Cp = C
@@ -579,24 +620,40 @@ int launch_score_d(const ScoreLaunch& s, cudaStream_t stream) {
                                                                             s.Bk, nK, s.kbar_hi, s.kbar_lo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
-  const size_t km_smem = kmeans_smem_bytes<D>();
-  static bool km_attr = false;
-  if (!km_attr) {
-    e = cudaFuncSetAttribute(kmeans_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(km_smem));
+  using KL = KmLayout<D>;
+  static int km_blocks_per_sm[2] = {0, 0};
+  if (!km_blocks_per_sm[0]) {
+    e = cudaFuncSetAttribute(kmeans_warp_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(KL::kAlloc));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(kmeans_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(km_smem));
+      e = cudaFuncSetAttribute(kmeans_warp_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(KL::kAlloc));
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&km_blocks_per_sm[0], kmeans_warp_kernel<D, 1>,
+                                                        kKmWarps * 32, KL::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&km_blocks_per_sm[1], kmeans_warp_kernel<D, 2>,
+                                                        kKmWarps * 32, KL::kAlloc);
     if (e != cudaSuccess) return static_cast<int>(e);
-    km_attr = true;
+    if (km_blocks_per_sm[0] < 1 || km_blocks_per_sm[1] < 1) return static_cast<int>(cudaErrorInvalidConfiguration);
   }
-  if (s.C <= 8)
-    kmeans_kernel<D, 1><<<dim3(s.G, BH), kScoreThreads, km_smem, stream>>>(
-        static_cast<const uint16_t*>(s.q), s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids, s.counts,
-        s.status);
-  else
-    kmeans_kernel<D, 2><<<dim3(s.G, BH), kScoreThreads, km_smem, stream>>>(
-        static_cast<const uint16_t*>(s.q), s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids, s.counts,
-        s.status);
+  {
+    // a persistent grid: every warp walks groups with a stride of the grid's warps
+    const long long items = static_cast<long long>(BH) * s.G;
+    const int per_sm = s.C <= 8 ? km_blocks_per_sm[0] : km_blocks_per_sm[1];
+    const long long want = (items + kKmWarps - 1) / kKmWarps;
+    const int grid = static_cast<int>(want < static_cast<long long>(s.num_sms) * per_sm
+                                          ? want
+                                          : static_cast<long long>(s.num_sms) * per_sm);
+    if (s.C <= 8)
+      kmeans_warp_kernel<D, 1><<<grid, kKmWarps * 32, KL::kAlloc, stream>>>(
+          static_cast<const uint16_t*>(s.q), BH, s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids,
+          s.counts, s.status);
+    else
+      kmeans_warp_kernel<D, 2><<<grid, kKmWarps * 32, KL::kAlloc, stream>>>(
+          static_cast<const uint16_t*>(s.q), BH, s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids,
+          s.counts, s.status);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
   int Cp = 1;
