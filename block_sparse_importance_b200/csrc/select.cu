@@ -109,7 +109,11 @@ __device__ __forceinline__ uint64_t block_scan_u64(uint64_t v, SelShared& sh, ui
   return before + inc - v;
 }
 
-// flags: bit0 exact, bit1 capped, bit2 drawn
+// CTA-per-row variant for rows longer than the warp kernel takes.  Thread t
+// owns the contiguous blocks [t E, (t+1) E) (E odd, so that the threads of a
+// warp reach distinct shared-memory banks), so every pass over the row is
+// thread-local and each scan is a local prefix plus one block-wide scan.
+// flags: bit0 exact, bit1 capped (or taken whole), bit2 drawn
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelShared sh;
@@ -124,6 +128,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   const int b = static_cast<int>(row / (static_cast<int64_t>(a.G) * a.H));
   const float* m = a.mass + row * nK;
   const int S = a.n_exact + a.n_sample;
+  const int E = ((nK + kSelThreads - 1) / kSelThreads) | 1;
+  const int i0 = min(nK, tid * E), i1 = min(nK, i0 + E);
 
   if (tid == 0) sh.bad = 0;
   __syncthreads();
@@ -147,8 +153,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += kSelThreads) sh.hist[i] = 0;
       __syncthreads();
-      for (int i = tid; i < nK; i += kSelThreads)
-        if ((key[i] & mask) == prefix) atomicAdd(&sh.hist[(key[i] >> shift) & 255u], 1u);
+      for (int i = i0; i < i1; ++i) {
+        const uint32_t k = key[i];
+        if ((k & mask) == prefix) atomicAdd(&sh.hist[(k >> shift) & 255u], 1u);
+      }
       __syncthreads();
       if (tid < 32) {
         // lane l owns bins [8l, 8l+8); suffix sums from the top bin down
@@ -184,34 +192,33 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
     }
     const uint32_t thr = prefix;
     const uint32_t take_ties = sh.remaining;
-    uint64_t carry = 0;
-    for (int base = 0; base < nK; base += kSelThreads) {
-      const int i = base + tid;
-      const uint32_t k = i < nK ? key[i] : 0u;
-      const bool tie = i < nK && k == thr;
-      uint64_t tot;
-      const uint64_t rank = carry + block_scan_u64(tie ? 1u : 0u, sh, &tot);
-      if (i < nK && (k > thr || (tie && rank < take_ties))) flag[i] = 1;
-      carry += tot;
+    uint64_t eq = 0;
+    for (int i = i0; i < i1; ++i) eq += key[i] == thr ? 1u : 0u;
+    uint64_t tot;
+    uint64_t rank = block_scan_u64(eq, sh, &tot);
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t k = key[i];
+      const bool tie = k == thr;
+      if (k > thr || (tie && rank < take_ties)) flag[i] = 1;
+      rank += tie ? 1u : 0u;
     }
-    __syncthreads();
   }
 
-  // ---- weights and capping over the rest
+  // ---- weights and capping over the rest (all per-block work is on the
+  // thread's own segment; only the totals cross threads)
   const int n_rest = nK - a.n_exact;
   int n_left = 0;
   uint64_t T = 0;
   if (a.n_sample >= n_rest) {
-    for (int i = tid; i < nK; i += kSelThreads)
+    for (int i = i0; i < i1; ++i)
       if (!(flag[i] & 1)) flag[i] |= 2;
-    __syncthreads();
   } else if (a.n_sample > 0) {
     uint32_t kmax = 0;
-    for (int i = tid; i < nK; i += kSelThreads)
+    for (int i = i0; i < i1; ++i)
       if (!(flag[i] & 1)) kmax = max(kmax, key[i]);
     kmax = block_max_u32(kmax, sh);
     const double mmax = static_cast<double>(__uint_as_float(kmax));
-    for (int i = tid; i < nK; i += kSelThreads) {
+    for (int i = i0; i < i1; ++i) {
       uint32_t w = 0;
       if (!(flag[i] & 1))
         w = mmax > 0.0 ? static_cast<uint32_t>(floor(static_cast<double>(__uint_as_float(key[i])) / mmax *
@@ -219,23 +226,21 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
                        : 1u;
       wq[i] = w;
     }
-    __syncthreads();
     int n_capped = 0;
     for (;;) {
       uint64_t t = 0;
-      for (int i = tid; i < nK; i += kSelThreads)
+      for (int i = i0; i < i1; ++i)
         if (!(flag[i] & 3)) t += wq[i];
       T = block_sum_u64(t, sh);
       n_left = a.n_sample - n_capped;
       uint64_t add = 0;
-      for (int i = tid; i < nK; i += kSelThreads)
+      for (int i = i0; i < i1; ++i)
         if (!(flag[i] & 3) && static_cast<uint64_t>(n_left) * wq[i] >= T) ++add;
       add = block_sum_u64(add, sh);  // all counts are taken before any flag changes
       if (add == 0) break;
-      for (int i = tid; i < nK; i += kSelThreads)
+      for (int i = i0; i < i1; ++i)
         if (!(flag[i] & 3) && static_cast<uint64_t>(n_left) * wq[i] >= T) flag[i] |= 2;
       n_capped += static_cast<int>(add);
-      __syncthreads();
     }
     if (n_left > 0) {
       const uint32_t U = static_cast<uint32_t>(
@@ -244,25 +249,33 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
       const uint64_t nl = static_cast<uint64_t>(n_left);
       const uint64_t ut_lo = static_cast<uint64_t>(U) * T;  // U T < 2^76
       const uint64_t ut_hi = __umul64hi(static_cast<uint64_t>(U), T);
-      // points of the systematic comb below x
-      auto below = [&](uint64_t x) -> uint64_t {
-        const uint64_t xn = x * nl;  // < 2^57
-        const uint64_t q = xn / T, r = xn - q * T;
-        const uint64_t r_hi = r >> 32, r_lo = r << 32;  // r * 2^32
-        const bool gt = r_hi > ut_hi || (r_hi == ut_hi && r_lo > ut_lo);
-        return q + (gt ? 1u : 0u);
+      // points of the comb below x: q + [r 2^32 > U T] with q = floor(x n' / T)
+      // and r = x n' - q T.  Walking x up by an uncapped weight (n' w < T)
+      // moves r up by n' w and needs at most one reduction by T, so only the
+      // start of each thread's segment takes a division.
+      auto above = [&](uint64_t r_) -> bool {
+        const uint64_t r_hi = r_ >> 32, r_lo = r_ << 32;
+        return r_hi > ut_hi || (r_hi == ut_hi && r_lo > ut_lo);
       };
-      uint64_t carry = 0;
-      for (int base = 0; base < nK; base += kSelThreads) {
-        const int i = base + tid;
-        const bool unc = i < nK && !(flag[i] & 3);
-        const uint64_t w = unc ? wq[i] : 0u;
-        uint64_t tot;
-        const uint64_t W_prev = carry + block_scan_u64(w, sh, &tot);
-        if (unc && below(W_prev + w) != below(W_prev)) flag[i] |= 4;
-        carry += tot;
+      uint64_t local = 0;
+      for (int i = i0; i < i1; ++i)
+        if (!(flag[i] & 3)) local += wq[i];
+      uint64_t tot;
+      const uint64_t xn0 = block_scan_u64(local, sh, &tot) * nl;
+      uint64_t q = xn0 / T, r = xn0 - q * T;
+      uint64_t f_prev = q + (above(r) ? 1u : 0u);
+      for (int i = i0; i < i1; ++i) {
+        if (!(flag[i] & 3)) {
+          r += static_cast<uint64_t>(wq[i]) * nl;
+          if (r >= T) {
+            r -= T;
+            ++q;
+          }
+          const uint64_t f = q + (above(r) ? 1u : 0u);
+          if (f != f_prev) flag[i] |= 4;
+          f_prev = f;
+        }
       }
-      __syncthreads();
     }
   }
 
@@ -270,32 +283,35 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   int32_t* out_idx = a.idx + row * S;
   float* out_lw = a.log_w + row * S;
   const double lnT = T > 0 ? log(static_cast<double>(T)) : 0.0;
-  uint64_t c_exact = 0, c_rest = static_cast<uint64_t>(a.n_exact);
-  for (int base = 0; base < nK; base += kSelThreads) {
-    const int i = base + tid;
-    const uint8_t f = i < nK ? flag[i] : 0;
-    uint64_t tot_e, tot_r;
-    const uint64_t pe = block_scan_u64((f & 1) ? 1u : 0u, sh, &tot_e);
-    const uint64_t pr = block_scan_u64((f & 6) ? 1u : 0u, sh, &tot_r);
-    if (f & 1) {
-      const uint64_t o = c_exact + pe;
-      if (o < static_cast<uint64_t>(a.n_exact)) {
-        out_idx[o] = i;
-        out_lw[o] = 0.0f;
-      }
-    } else if (f & 6) {
-      const uint64_t o = c_rest + pr;
-      if (o < static_cast<uint64_t>(S)) {
-        out_idx[o] = i;
-        out_lw[o] = (f & 4) ? static_cast<float>(lnT - log(static_cast<double>(static_cast<uint64_t>(n_left) * wq[i])))
-                            : 0.0f;
-      }
-    }
-    c_exact += tot_e;
-    c_rest += tot_r;
+  uint64_t ne = 0, nr = 0;
+  for (int i = i0; i < i1; ++i) {
+    const uint8_t f = flag[i];
+    ne += (f & 1) ? 1u : 0u;
+    nr += (!(f & 1) && (f & 6)) ? 1u : 0u;
   }
+  uint64_t tot;
+  const uint64_t pre = block_scan_u64((ne << 32) | nr, sh, &tot);  // both counts < 2^32
+  uint64_t pe = pre >> 32, pr = static_cast<uint64_t>(a.n_exact) + (pre & 0xFFFFFFFFull);
+  for (int i = i0; i < i1; ++i) {
+    const uint8_t f = flag[i];
+    if (f & 1) {
+      if (pe < static_cast<uint64_t>(a.n_exact)) {
+        out_idx[pe] = i;
+        out_lw[pe] = 0.0f;
+      }
+      ++pe;
+    } else if (f & 6) {
+      if (pr < static_cast<uint64_t>(S)) {
+        out_idx[pr] = i;
+        out_lw[pr] = (f & 4) ? static_cast<float>(lnT - log(static_cast<double>(static_cast<uint64_t>(n_left) * wq[i])))
+                             : 0.0f;
+      }
+      ++pr;
+    }
+  }
+  const uint64_t tot_e = tot >> 32, tot_r = tot & 0xFFFFFFFFull;
   if (tid == 0) {
-    if (sh.bad || c_exact != static_cast<uint64_t>(a.n_exact) || c_rest != static_cast<uint64_t>(S))
+    if (sh.bad || tot_e != static_cast<uint64_t>(a.n_exact) || tot_e + tot_r != static_cast<uint64_t>(S))
       atomicCAS(a.status, 0, kStatusDeviceCheck);
   }
 }

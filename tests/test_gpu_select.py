@@ -38,7 +38,10 @@ def _compare(isa, mass, ne, ns, seed, H, G, nK, Bk=64):
 
 @pytest.mark.parametrize("kind", ["lognormal", "ties", "spiky", "zeros"])
 @pytest.mark.parametrize("nK,ne,ns", [(64, 4, 4), (37, 0, 9), (1182, 39, 79), (512, 16, 35), (300, 0, 0 + 1),
-                                      (200, 150, 50)])
+                                      (200, 150, 50),
+                                      # rows longer than 2048 blocks take the CTA-per-row kernel
+                                      (2049, 0, 30), (3000, 40, 80), (7425, 248, 496), (5000, 4990, 5),
+                                      (4100, 100, 4000)])
 def test_select_bit_exact(isa, kind, nK, ne, ns):
     rng = np.random.default_rng(nK + ne)
     H, G = 2, 8
