@@ -59,6 +59,24 @@ def attn_traffic(workload, heads):
     return ATTN_TRAFFIC["bytes_per_head"] * heads
 
 
+def reduce_max_over_ranks(values, device):
+    """Max of each value over all ranks (identity with one process): the job's
+    time is its slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_throughput(world: int, flops_per_rank: float, ms: float) -> float:
+    """Whole-job TFLOP/s: every rank computes its own layer (weak scaling), so
+    the job does world x flops_per_rank in the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -298,12 +316,9 @@ def main():
     attn_ms = sum(e[0].elapsed_time(e[1]) for e in attn_ev) / args.steps
     score_ms = sum(e[2].elapsed_time(e[3]) for e in attn_ev) / args.steps
     select_ms = sum(e[3].elapsed_time(e[0]) for e in attn_ev) / args.steps
-    if world > 1:
-        tt = torch.tensor([elapsed_ms, attn_ms, score_ms, select_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms, attn_ms, score_ms, select_ms = (float(x) for x in tt)
+    elapsed_ms, attn_ms, score_ms, select_ms = reduce_max_over_ranks([elapsed_ms, attn_ms, score_ms, select_ms], dev)
     ms_step = elapsed_ms / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = job_throughput(world, flops, ms_step)
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
@@ -356,13 +371,9 @@ def main():
             isa.pipeline_host(qh, kh, vh, oh, lay, p, arena, ctx=ctx, device=local)
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt[0])
+        e_ms = reduce_max_over_ranks([e0.elapsed_time(e1) / n_e2e], dev)[0]
         nbytes = q.numel() * q.element_size()
-        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+        e2e = {"value": job_throughput(world, flops, e_ms), "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
                "api": "isa_pipeline_host (pinned host buffers)"}
         del arena
