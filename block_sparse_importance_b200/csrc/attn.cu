@@ -514,8 +514,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // pass 2: P = exp2(z - max) as bf16 pairs; chunk c's 8 packed columns
         // land on columns 8c.. of this half's S, which earlier chunks already read
+        // (the scale-and-shift and the running sums use paired fp32 arithmetic:
+        // one instruction for two elements)
         {
-          float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          uint64_t ls2[2] = {0ull, 0ull};  // (even, odd) partial sums; zero bits are (0.0f, 0.0f)
+          const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
           uint32_t sv[2][16];
           tmem_ld16(lane_base + col_s, sv[0]);
           tmem_wait_ld();
@@ -525,23 +528,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t* v = sv[c & 1];
             const float bm = __shfl_sync(0xffffffffu, c_bias, c) - m_used;
             const int nv = __shfl_sync(0xffffffffu, c_valid, c);
+            const uint64_t bm2 = f2_pack(bm, bm);
             uint32_t pk[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              float x0 = fmaf(__uint_as_float(v[2 * i]), a.scale_log2, bm);
-              float x1 = fmaf(__uint_as_float(v[2 * i + 1]), a.scale_log2, bm);
+              float x0, x1;
+              f2_unpack(fma_f32x2(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), sc2, bm2), x0,
+                        x1);
               if (partial) {
                 x0 = 2 * i < nv ? x0 : -INFINITY;
                 x1 = 2 * i + 1 < nv ? x1 : -INFINITY;
               }
               const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-              ls[i & 3] += p0 + p1;
+              ls2[i & 1] = add_f32x2(ls2[i & 1], f2_pack(p0, p1));
               pk[i] = pack_bf16x2(p0, p1);
             }
             tmem_st8(lane_base + col_s + 8 * c, pk);
             if (c < 3) tmem_wait_ld();
           }
-          l_sum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          float s0, s1, s2, s3;
+          f2_unpack(ls2[0], s0, s1);
+          f2_unpack(ls2[1], s2, s3);
+          l_sum += (s0 + s1) + (s2 + s3);
         }
         tmem_wait_st();
         tc_fence_before();
