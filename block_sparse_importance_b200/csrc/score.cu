@@ -471,28 +471,35 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     }
   } else if (warp == 5) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // The whole warp runs the loop and waits; one elected lane issues.  The
+    // shared-memory descriptors are built once and advanced by adds to their
+    // start-address field (addresses stay below 2^18: no carry out of it).
+    {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0);
+      const uint64_t da_hi = smem_desc_sw128(base + L::kAHi, 16, 1024);
+      const uint64_t da_lo = smem_desc_sw128(base + L::kALo, 16, 1024);
+      const uint64_t db = smem_desc_sw128(base + L::kRing, 16, 1024);
       for (int i = 0; i < n_items; ++i) {
         const uint32_t slot = i % kMassRing, buf = i & 1;
-        if (!mbar_wait(bar(L::kBarFull + slot), (i / kMassRing) & 1u, abort_flag, kWaitTimeoutNs)) break;
-        if (!mbar_wait(bar(L::kBarSFree + buf), ((i >> 1) & 1u) ^ 1u, abort_flag, kWaitTimeoutNs)) break;
+        if (!mbar_wait_warp(bar(L::kBarFull + slot), (i / kMassRing) & 1u, abort_flag, kWaitTimeoutNs)) break;
+        if (!mbar_wait_warp(bar(L::kBarSFree + buf), ((i >> 1) & 1u) ^ 1u, abort_flag, kWaitTimeoutNs)) break;
         tc_fence_after();
-        const uint32_t b_hi = base + L::kRing + slot * L::kStage, b_lo = b_hi + L::kTile;
-        const uint32_t a_hi = base + L::kAHi, a_lo = base + L::kALo;
+        const uint64_t b_hi = db + ((slot * L::kStage) >> 4), b_lo = b_hi + (L::kTile >> 4);
         const uint32_t d = tmem + buf * 128;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * L::kChunk + (k & 3) * 32;
-          mma_ss(d, smem_desc_sw128(a_hi + off, 16, 1024), smem_desc_sw128(b_hi + off, 16, 1024), idesc,
-                 k > 0 ? 1u : 0u);
-          mma_ss(d, smem_desc_sw128(a_hi + off, 16, 1024), smem_desc_sw128(b_lo + off, 16, 1024), idesc, 1u);
-          mma_ss(d, smem_desc_sw128(a_lo + off, 16, 1024), smem_desc_sw128(b_hi + off, 16, 1024), idesc, 1u);
+          const uint64_t off = ((k >> 2) * L::kChunk + (k & 3) * 32) >> 4;
+          if (elect_one()) mma_ss(d, da_hi + off, b_hi + off, idesc, k > 0 ? 1u : 0u);
+          if (elect_one()) mma_ss(d, da_hi + off, b_lo + off, idesc, 1u);
+          if (elect_one()) mma_ss(d, da_lo + off, b_hi + off, idesc, 1u);
         }
-        tc_commit(bar(L::kBarEmpty + slot));
-        tc_commit(bar(L::kBarSFull + buf));
+        if (elect_one()) {
+          tc_commit(bar(L::kBarEmpty + slot));
+          tc_commit(bar(L::kBarSFull + buf));
+        }
       }
-      tc_commit(bar(L::kBarFinal));
+      if (elect_one()) tc_commit(bar(L::kBarFinal));
+      __syncwarp();
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(bar(L::kBarFinal), 0))
         if (global_timer_ns() - t0 > 200000000ull) break;
