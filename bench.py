@@ -43,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Q, K, V and O all scale with the head count.  The figure holds only for the
 # kernel source whose SHA-256 starts with the recorded prefix; for any other
 # source (or workload) the roofline reports traffic as null.
-ATTN_TRAFFIC = {"workload": "wan14_10", "src_sha256_prefix": "8a4912f9f9c6eb15", "bytes_per_head": 307.8e6 / 4}
+ATTN_TRAFFIC = {"workload": "wan14_10", "src_sha256_prefix": "586c989f603b9d27", "bytes_per_head": 310.3e6 / 4}
 
 
 def attn_traffic(workload, heads):
