@@ -41,19 +41,29 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch, per head, from an ncu capture of the wan14_10 layer cut to 4 heads.
 # Q, K, V and O all scale with the head count.  The figure holds only for the
-# kernel source whose SHA-256 starts with the recorded prefix; for any other
-# source (or workload) the roofline reports traffic as null.
-ATTN_TRAFFIC = {"workload": "wan14_10", "src_sha256_prefix": "586c989f603b9d27", "bytes_per_head": 310.3e6 / 4}
+# kernel source whose code (comments and blank lines removed) has a SHA-256
+# starting with the recorded prefix; for any other source (or workload) the
+# roofline reports traffic as null.
+ATTN_TRAFFIC = {"workload": "wan14_10", "src_sha256_prefix": "0ac1e018455c7ae4", "bytes_per_head": 310.3e6 / 4}
+
+
+def attn_code_digest(text: str) -> str:
+    """SHA-256 of a CUDA source with // comments and blank lines removed."""
+    import hashlib
+    import re
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()
 
 
 def attn_traffic(workload, heads):
     import hashlib
     src = os.path.join(ROOT, "block_sparse_importance_b200", "csrc", "attn.cu")
     try:
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+        with open(src) as f:
+            code = attn_code_digest(f.read())
     except OSError:
         return None
+    sha = code
     if workload != ATTN_TRAFFIC["workload"] or not sha.startswith(ATTN_TRAFFIC["src_sha256_prefix"]):
         return None
     return ATTN_TRAFFIC["bytes_per_head"] * heads

@@ -8,22 +8,25 @@
 // value blocks much smaller than a tile are gathered into full tensor-core
 // tiles).
 //
-// Kernel design (one persistent CTA per SM, 10 warps):
+// Kernel design (one persistent CTA per SM, 18 warps):
 //   * a work item is one query tile of <= 128 rows of one (batch, head,
 //     group); a CTA takes items in pairs (A, B) and ping-pongs them so the
 //     softmax of one tile overlaps the tensor-core work of the other;
-//   * warp 8 (producer) streams K and V tiles of 128 rows through a 4-stage
+//   * warp 16 (producer) streams K and V tiles of 128 rows through a 4-stage
 //     shared-memory ring with TMA, gathering every plan block of k_block rows
 //     (16..128) into its place in the tile (one box per block and 64-column
 //     chunk, 128-byte swizzle, out-of-range rows zero-filled);
-//   * warp 9 (MMA) issues tcgen05.mma: S = Q K^T into TMEM (both operands
-//     K-major in shared memory), then O += P V with P read from TMEM and V
-//     MN-major in shared memory, fp32 accumulation in TMEM;
-//   * warps 0-3 / 4-7 (softmax, one thread per query row = TMEM lane) read S,
-//     add scale*s + log_w(block) (log2 units), mask invalid rows, keep an
-//     online max that is raised (and O rescaled in TMEM) only when it grows
-//     by more than 2^8, write P = exp2(z - max) as bf16 over S's columns, and
-//     finally normalise O and store bf16 rows and the log-sum-exp.
+//   * warp 17 (MMA) runs converged and issues tcgen05.mma through an elected
+//     lane: S = Q K^T into TMEM (both operands K-major in shared memory),
+//     then O += P V with P read from TMEM and V MN-major in shared memory,
+//     fp32 accumulation in TMEM;
+//   * warps 0-7 / 8-15 (softmax of tile A / B): two warps per 32-row TMEM
+//     lane slice, each over one 64-column half of the row.  They read S, add
+//     scale*s + log_w(block) (log2 units), mask invalid rows, agree on the
+//     row max through shared memory, keep an online max that is raised (and
+//     their half of O rescaled in TMEM) only when it grows by more than 2^8,
+//     write P = exp2(z - max) as bf16 over S's columns, and finally normalise
+//     their half of O and store bf16 rows and the log-sum-exp.
 // When both tiles of a pair read the same plan (dense mode, or two tiles of
 // one cluster) the K/V stream is loaded once and used by both.
 // Every barrier wait is bounded; on a timeout the CTA stops issuing work,
