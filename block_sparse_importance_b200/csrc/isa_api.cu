@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "isa.h"
 #include "isa_internal.h"
@@ -20,6 +21,7 @@ struct isa_context {
   int* d_status;
   uint64_t wait_timeout_ns;  // 0: the kernels' default
   int stall_attention;       // failure-detection test hook
+  cudaStream_t copy_in, copy_out;  // isa_pipeline_host's copy streams (made on first use)
   char last_error[512];
 };
 
@@ -155,7 +157,7 @@ isa_status do_score(isa_context* ctx, const isa_shape* s, const void* q, const v
 }
 
 isa_status do_select(isa_context* ctx, const isa_shape* s, const float* mass, int32_t ne, int32_t ns, uint64_t seed,
-                     int32_t* idx, float* log_w, cudaStream_t st) {
+                     int32_t* idx, float* log_w, cudaStream_t st, int h_base = 0, int b_base = 0) {
   ISA_TRY(check_ptr(ctx, mass, "mass", 4));
   ISA_TRY(check_ptr(ctx, idx, "idx", 4));
   ISA_TRY(check_ptr(ctx, log_w, "log_w", 4));
@@ -170,6 +172,8 @@ isa_status do_select(isa_context* ctx, const isa_shape* s, const float* mass, in
   l.nK = nK;
   l.n_exact = ne;
   l.n_sample = ns;
+  l.h_base = h_base;
+  l.b_base = b_base;
   l.seed = seed;
   l.mass = mass;
   l.idx = idx;
@@ -237,7 +241,7 @@ size_t pipeline_bytes(const isa_shape* s, const isa_params* p) {
 
 isa_status do_pipeline(isa_context* ctx, const isa_shape* s, const isa_params* p, const void* q, const void* k,
                        const void* v, void* out, float* lse, int32_t* plan_idx, float* plan_lw, void* ws,
-                       size_t ws_bytes, cudaStream_t st) {
+                       size_t ws_bytes, cudaStream_t st, int h_base = 0, int b_base = 0) {
   if (!p) return fail(ctx, ISA_ERR_INVALID_ARG, "params is NULL");
   if (p->n_clusters < 1 || p->n_clusters > 16) return fail(ctx, ISA_ERR_INVALID_ARG, "n_clusters must be 1..16");
   const size_t need = pipeline_bytes(s, p);
@@ -259,7 +263,7 @@ isa_status do_pipeline(isa_context* ctx, const isa_shape* s, const isa_params* p
   w += round_up(rows * S * 4);
   void* aws = w;
   ISA_TRY(do_score(ctx, s, q, k, p->n_clusters, p->n_iters, mass, nullptr, nullptr, sws, score_ws, st));
-  ISA_TRY(do_select(ctx, s, mass, p->n_exact, p->n_sample, p->seed, idx, lw, st));
+  ISA_TRY(do_select(ctx, s, mass, p->n_exact, p->n_sample, p->seed, idx, lw, st, h_base, b_base));
   return do_attention(ctx, s, q, k, v, idx, lw, static_cast<int32_t>(S), out, lse, aws, attn_ws_bytes(s), false, st);
 }
 
@@ -303,6 +307,8 @@ void isa_destroy(isa_context* ctx) {
   if (!ctx) return;
   DeviceGuard g(ctx->device);
   cudaFree(ctx->d_status);
+  if (ctx->copy_in) cudaStreamDestroy(ctx->copy_in);
+  if (ctx->copy_out) cudaStreamDestroy(ctx->copy_out);
   delete ctx;
 }
 
@@ -426,15 +432,88 @@ isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, const isa
   const size_t bytes = static_cast<size_t>(shape->batch) * shape->heads * shape->seq_len * shape->head_dim * 2;
   const size_t t = round_up(bytes);
   char* w = static_cast<char*>(workspace);
-  void *dq = w, *dk = w + t, *dv = w + 2 * t, *dout = w + 3 * t;
-  cudaError_t e = cudaMemcpyAsync(dq, q_host, bytes, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k_host, bytes, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v_host, bytes, cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) return fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host copy in: %s", cudaGetErrorString(e));
-  ISA_TRY(do_pipeline(ctx, shape, params, dq, dk, dv, dout, nullptr, nullptr, nullptr, w + 4 * t, need - 4 * t, st));
-  e = cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, st);
-  if (e != cudaSuccess) return fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host copy out: %s", cudaGetErrorString(e));
-  return ISA_OK;
+  char *dq = w, *dk = w + t, *dv = w + 2 * t, *dout = w + 3 * t;
+  // The layer runs in chunks of heads so that copies overlap the compute:
+  // chunk i's inputs go up on one copy stream while chunk i-1 computes on
+  // `stream` and chunk i-2's output comes down on another.  Heads are
+  // independent, and the selector keys its uniform by the global head and
+  // batch index, so the result is the one isa_pipeline gives on the whole
+  // layer.
+  if (!ctx->copy_in && cudaStreamCreateWithFlags(&ctx->copy_in, cudaStreamNonBlocking) != cudaSuccess)
+    return fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host: cannot create a copy stream");
+  if (!ctx->copy_out && cudaStreamCreateWithFlags(&ctx->copy_out, cudaStreamNonBlocking) != cudaSuccess)
+    return fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host: cannot create a copy stream");
+  const int H = shape->heads;
+  const int hc = (H + 7) / 8;  // heads per chunk: up to 8 chunks per batch entry
+  const size_t head_bytes = static_cast<size_t>(shape->seq_len) * shape->head_dim * 2;
+  std::vector<cudaEvent_t> evs;
+  auto new_event = [&](cudaEvent_t* ev) -> bool {
+    if (cudaEventCreateWithFlags(ev, cudaEventDisableTiming) != cudaSuccess) return false;
+    evs.push_back(*ev);
+    return true;
+  };
+  auto release = [&]() {
+    for (cudaEvent_t ev : evs) cudaEventDestroy(ev);  // pending records complete first
+  };
+  isa_status result = ISA_OK;
+  cudaError_t e = cudaSuccess;
+  cudaEvent_t start;
+  // nothing may overwrite the arena before earlier work on `stream` is done
+  if (!new_event(&start) || (e = cudaEventRecord(start, st)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(ctx->copy_in, start, 0)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(ctx->copy_out, start, 0)) != cudaSuccess) {
+    release();
+    return fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host: event setup failed");
+  }
+  for (int b = 0; b < shape->batch && result == ISA_OK; ++b) {
+    for (int h0 = 0; h0 < H && result == ISA_OK; h0 += hc) {
+      const int nh = H - h0 < hc ? H - h0 : hc;
+      const size_t off = (static_cast<size_t>(b) * H + h0) * head_bytes, len = static_cast<size_t>(nh) * head_bytes;
+      cudaEvent_t in_done, comp_done;
+      if (!new_event(&in_done) || !new_event(&comp_done)) {
+        result = fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host: cannot create an event");
+        break;
+      }
+      e = cudaMemcpyAsync(dq + off, static_cast<const char*>(q_host) + off, len, cudaMemcpyHostToDevice, ctx->copy_in);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dk + off, static_cast<const char*>(k_host) + off, len, cudaMemcpyHostToDevice,
+                            ctx->copy_in);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dv + off, static_cast<const char*>(v_host) + off, len, cudaMemcpyHostToDevice,
+                            ctx->copy_in);
+      if (e == cudaSuccess) e = cudaEventRecord(in_done, ctx->copy_in);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(st, in_done, 0);
+      if (e != cudaSuccess) {
+        result = fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host copy in: %s", cudaGetErrorString(e));
+        break;
+      }
+      isa_shape sub = *shape;
+      sub.batch = 1;
+      sub.heads = nh;
+      result = do_pipeline(ctx, &sub, params, dq + off, dk + off, dv + off, dout + off, nullptr, nullptr, nullptr,
+                           w + 4 * t, need - 4 * t, st, h0, b);
+      if (result != ISA_OK) break;
+      e = cudaEventRecord(comp_done, st);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->copy_out, comp_done, 0);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(static_cast<char*>(out_host) + off, dout + off, len, cudaMemcpyDeviceToHost,
+                            ctx->copy_out);
+      if (e != cudaSuccess) result = fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host copy out: %s", cudaGetErrorString(e));
+    }
+  }
+  // `stream` completes only after the last output copy (and, on an error, after
+  // whatever was enqueued on the copy streams)
+  cudaEvent_t fin_in, fin_out;
+  if (new_event(&fin_in) && new_event(&fin_out)) {
+    cudaEventRecord(fin_in, ctx->copy_in);
+    cudaEventRecord(fin_out, ctx->copy_out);
+    cudaStreamWaitEvent(st, fin_in, 0);
+    cudaStreamWaitEvent(st, fin_out, 0);
+  } else if (result == ISA_OK) {
+    result = fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host: cannot create an event");
+  }
+  release();
+  return result;
 }
 
 }  // extern "C"

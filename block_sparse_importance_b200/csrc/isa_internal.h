@@ -47,6 +47,7 @@ int launch_attention(const AttnLaunch& a, const void* q, const void* k, const vo
 // -------------------------------------------------------------- selector
 struct SelectLaunch {
   int B, H, G, nK, n_exact, n_sample;
+  int h_base, b_base;  // head and batch index of the launch's first row in the whole tensor
   uint64_t seed;
   const float* mass;
   int32_t* idx;

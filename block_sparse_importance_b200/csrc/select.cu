@@ -244,7 +244,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
     }
     if (n_left > 0) {
       const uint32_t U = static_cast<uint32_t>(
-          philox_word0(static_cast<uint32_t>(g), static_cast<uint32_t>(h), static_cast<uint32_t>(b), 0, a.seed, 0) >>
+          philox_word0(static_cast<uint32_t>(g), static_cast<uint32_t>(h + a.h_base), static_cast<uint32_t>(b + a.b_base), 0,
+                       a.seed, 0) >>
           32);
       const uint64_t nl = static_cast<uint64_t>(n_left);
       const uint64_t ut_lo = static_cast<uint64_t>(U) * T;  // U T < 2^76
@@ -465,7 +466,8 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
     }
     if (n_left > 0) {
       const uint32_t U = static_cast<uint32_t>(
-          philox_word0(static_cast<uint32_t>(g), static_cast<uint32_t>(h), static_cast<uint32_t>(b), 0, a.seed, 0) >>
+          philox_word0(static_cast<uint32_t>(g), static_cast<uint32_t>(h + a.h_base), static_cast<uint32_t>(b + a.b_base), 0,
+                       a.seed, 0) >>
           32);
       const uint64_t nl = static_cast<uint64_t>(n_left);
       const uint64_t ut_lo = static_cast<uint64_t>(U) * T;  // U T < 2^76

@@ -217,8 +217,15 @@ ISA_API isa_status isa_pipeline(isa_context* ctx, const isa_shape* shape, const 
  * device arena, runs the pipeline, and copies the output back to out_host
  * ([B,H,N,d] bf16).  The arena holds Q, K, V, O and the pipeline workspace:
  * isa_pipeline_host_workspace_bytes bytes.  shape->q_offsets stays a device
- * pointer.  Enqueues everything on `stream`; out_host is valid after the
- * stream is synchronised.
+ * pointer.  The layer runs in chunks of heads (up to 8 per batch entry) so
+ * that the copies overlap the compute: the inputs go up and the outputs come
+ * down on two copy streams the context owns, the compute runs on `stream`,
+ * and events order them.  The result equals isa_pipeline on the whole layer
+ * (the selector's uniform is keyed by the global head and batch index).
+ * Returns after enqueueing; `stream` completes only after the last output
+ * copy, so out_host is valid once `stream` is synchronised.  Work already on
+ * `stream` is finished before the arena is overwritten.  Calls that share a
+ * context share its copy streams.
  * ------------------------------------------------------------------------- */
 ISA_API size_t isa_pipeline_host_workspace_bytes(const isa_shape* shape, const isa_params* params);
 ISA_API isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, const isa_params* params,
