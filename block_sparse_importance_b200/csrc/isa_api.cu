@@ -444,7 +444,7 @@ isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, const isa
   if (!ctx->copy_out && cudaStreamCreateWithFlags(&ctx->copy_out, cudaStreamNonBlocking) != cudaSuccess)
     return fail(ctx, ISA_ERR_CUDA, "isa_pipeline_host: cannot create a copy stream");
   const int H = shape->heads;
-  const int hc = (H + 7) / 8;  // heads per chunk: up to 8 chunks per batch entry
+  const int hc = (H + 15) / 16;  // heads per chunk: up to 16 chunks per batch entry
   const size_t head_bytes = static_cast<size_t>(shape->seq_len) * shape->head_dim * 2;
   std::vector<cudaEvent_t> evs;
   auto new_event = [&](cudaEvent_t* ev) -> bool {

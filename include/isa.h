@@ -217,7 +217,7 @@ ISA_API isa_status isa_pipeline(isa_context* ctx, const isa_shape* shape, const 
  * device arena, runs the pipeline, and copies the output back to out_host
  * ([B,H,N,d] bf16).  The arena holds Q, K, V, O and the pipeline workspace:
  * isa_pipeline_host_workspace_bytes bytes.  shape->q_offsets stays a device
- * pointer.  The layer runs in chunks of heads (up to 8 per batch entry) so
+ * pointer.  The layer runs in chunks of heads (up to 16 per batch entry) so
  * that the copies overlap the compute: the inputs go up and the outputs come
  * down on two copy streams the context owns, the compute runs on `stream`,
  * and events order them.  The result equals isa_pipeline on the whole layer
