@@ -14,6 +14,9 @@ roofline     the attention kernel (dominant): computed FLOPs per launch / its
              event-timed duration, against the measured bf16 tensor peak.
 e2e          the same metric through isa_pipeline_host: pinned host Q/K/V in,
              host O out, copies inside the timed region.
+plan_reuse_ms_per_call
+             ms per attention call when one plan serves r calls (score and
+             select once per r), measured for r = 2, 4, 8; outside the step.
 Multi-GPU: one process per GPU (torchrun); every rank runs its own layer
 (weak scaling, no data-path collective); time = max over ranks.
 """
@@ -349,6 +352,21 @@ def main():
     for v_ in stages.values():
         v_["frac_hbm"] = v_["gbs"] / hbm
 
+    # plan reuse across calls (a plan made once serves r attention calls):
+    # measured ms per attention call, score and select included once per r
+    plan_reuse = {}
+    for r in (2, 4, 8):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(2):
+            isa.score(q, k, lay, w.n_clusters, w.n_iters, mass=mass, workspace=sws, ctx=ctx)
+            isa.select(mass, lay, w.n_exact, w.n_sample, w.seed, idx=idx, log_w=lw, ctx=ctx)
+            for _ in range(r):
+                isa.attention(q, k, v, idx, lw, lay, out=out, workspace=aws, ctx=ctx)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        plan_reuse[str(r)] = e0.elapsed_time(e1) / (2 * r)
+
     # dense limit, same tensors (context for the speedup analogue)
     dense_ms = None
     if rank == 0:
@@ -403,7 +421,8 @@ def main():
                 "dense_attention_ms": dense_ms,
                 "sparse_vs_dense": (dense_ms / attn_ms) if dense_ms else None,
                 "computed_tflop_per_step": flops / 1e12,
-                "roofline": roofline, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "stages": stages, "plan_reuse_ms_per_call": plan_reuse,
+                "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -157,12 +157,10 @@ __device__ __forceinline__ void set_status(int* status, int code) { atomicCAS(st
 
 // Wait that ignores the abort flag, used only to drain in-flight copies.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-  volatile int never = 0;
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (global_timer_ns() - t0 > 200000000ull) break;
   }
-  (void)never;
 }
 
 template <int D>

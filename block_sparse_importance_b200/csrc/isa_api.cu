@@ -1,7 +1,8 @@
 // C ABI of libisa.so (declared in include/isa.h): argument checks, the
 // per-context device status word, workspace carving and kernel launches.
-// The library allocates nothing in a call path; every device buffer belongs
-// to the caller.
+// The library allocates no device memory in a call path; every device buffer
+// belongs to the caller.  (isa_pipeline_host creates two copy streams on its
+// first call, kept by the context, and a few events per call.)
 
 #include <cuda_runtime.h>
 
