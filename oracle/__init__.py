@@ -59,6 +59,10 @@ def _load():
             lib.ref_select_row.restype = i32
             lib.ref_select.argtypes = [P, i32, i32, i32, i32, i32, i32, u64, P, P, P, i32]
             lib.ref_select.restype = i32
+            lib.ref_top_p_count.argtypes = [P, i32, f64, i32, P]
+            lib.ref_top_p_count.restype = i32
+            lib.ref_select_top_p.argtypes = [P, i32, i32, i32, i32, f64, i32, u64, P, P, P, P, i32]
+            lib.ref_select_top_p.restype = i32
             lib.ref_attention.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, i32, P, P, i32, f64,
                                           P, i32, P, P, i32]
             lib.ref_dense_attention.argtypes = [P, P, P, i32, i32, f64, P, i32, P, P, i32]
@@ -178,6 +182,33 @@ def select(mass: np.ndarray, n_exact: int, n_sample: int, seed: int, threads: in
     if st != 0:
         raise ValueError("ref_select failed with %d" % st)
     return idx, lw, bool(bad[0])
+
+
+def top_p_count(mass_row: np.ndarray, p: float, S: int):
+    """Exact-set size of one row under the top-p rule (see ref_top_p_count).
+    Returns (k_e, bad)."""
+    m = _c(mass_row, np.float32)
+    bad = np.zeros(1, np.int32)
+    k = _load().ref_top_p_count(_p(m), m.shape[0], ctypes.c_double(p), S, _p(bad))
+    if k < 0:
+        raise ValueError("ref_top_p_count: bad arguments")
+    return int(k), bool(bad[0])
+
+
+def select_top_p(mass: np.ndarray, p: float, S: int, seed: int, threads: int = 0):
+    """mass: [B, H, G, nK] fp32 -> (idx [B,H,G,S] i32, log_w [B,H,G,S] f32,
+    k_e [B,H,G] i32, bad) under the top-p rule."""
+    m = _c(mass, np.float32)
+    B, H, G, nK = m.shape
+    idx = np.zeros((B, H, G, S), np.int32)
+    lw = np.zeros((B, H, G, S), np.float32)
+    ke = np.zeros((B, H, G), np.int32)
+    bad = np.zeros(1, np.int32)
+    st = _load().ref_select_top_p(_p(m), B, H, G, nK, ctypes.c_double(p), S, ctypes.c_uint64(seed), _p(idx),
+                                  _p(lw), _p(ke), _p(bad), threads)
+    if st != 0:
+        raise ValueError("ref_select_top_p failed with %d" % st)
+    return idx, lw, ke, bool(bad[0])
 
 
 def attention(q, k, v, offsets, k_block: int, idx, log_w, scale: float, groups, threads: int = 0):

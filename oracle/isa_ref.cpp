@@ -423,6 +423,91 @@ int32_t ref_select(const float* mass, int32_t B, int32_t H, int32_t G, int32_t n
 }
 
 // ---------------------------------------------------------------------------
+// Exact-set size from a share of the mass (the top-p rule of "iCATS", Method
+// summary: sparsity set by the share p of attention mass kept).  Reading: the
+// exact set is the shortest head of the blocks in descending mass order (ties
+// to the lower block) whose mass reaches the share p of the row's total; it is
+// capped at the plan size S, and the rest of the budget, S - k_e, is sampled
+// as above.  In exact integers, so that every implementation agrees:
+//   q_b = floor(m_b / m_max * 2^31) in IEEE fp64 for m_b > 0, else 0
+//         (m_max = the row's largest mass; all q are 0 when it is 0);
+//   target = ceil(p * sum_b q_b) in fp64 (the sum is below 2^45: exact);
+//   k_e = min(S, smallest k with q_(1) + ... + q_(k) >= target).
+// A row of zeros has target 0 and k_e = 0.  Non-finite masses count as 0
+// (and set *bad).  Returns k_e, or -1 on bad arguments.
+// ---------------------------------------------------------------------------
+int32_t ref_top_p_count(const float* mass, int32_t nK, double p, int32_t S, int32_t* bad) {
+  if (nK < 1 || S < 0 || S > nK || !(p > 0.0) || p > 1.0) return -1;
+  std::vector<uint32_t> key(nK);
+  uint32_t kmax = 0;
+  for (int32_t b = 0; b < nK; ++b) {
+    const float m = mass[b];
+    if (!std::isfinite(m)) {
+      if (bad) *bad = 1;
+      key[b] = 0;
+    } else {
+      key[b] = m > 0.0f ? float_bits(m) : 0u;
+    }
+    kmax = std::max(kmax, key[b]);
+  }
+  float mmax_f;
+  std::memcpy(&mmax_f, &kmax, 4);
+  const double mmax = static_cast<double>(mmax_f);
+  std::vector<uint64_t> q(nK, 0);
+  uint64_t total = 0;
+  for (int32_t b = 0; b < nK; ++b) {
+    if (key[b] != 0 && mmax > 0.0) {
+      float f;
+      std::memcpy(&f, &key[b], 4);
+      q[b] = static_cast<uint64_t>(std::floor(static_cast<double>(f) / mmax * 2147483648.0));
+    }
+    total += q[b];
+  }
+  const uint64_t target = static_cast<uint64_t>(std::ceil(p * static_cast<double>(total)));
+  // descending key, ties to the lower block
+  std::vector<int32_t> order(nK);
+  for (int32_t b = 0; b < nK; ++b) order[b] = b;
+  std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) { return key[x] > key[y]; });
+  int32_t k = 0;
+  uint64_t cum = 0;
+  while (cum < target && k < nK) cum += q[order[k++]];
+  return std::min(k, S);
+}
+
+// All rows of a [B, H, G, nK] mass tensor under the top-p rule: the exact-set
+// size of each row (k_e, [B, H, G]) and the plan with n_exact = k_e and
+// n_sample = S - k_e (idx / log_w: [B, H, G, S]); uniforms as ref_select.
+int32_t ref_select_top_p(const float* mass, int32_t B, int32_t H, int32_t G, int32_t nK, double p, int32_t S,
+                         uint64_t seed, int32_t* idx, float* log_w, int32_t* k_e, int32_t* bad,
+                         int32_t nthreads) {
+  const int64_t rows = static_cast<int64_t>(B) * H * G;
+  int32_t status = 0;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel for schedule(dynamic) reduction(min : status)
+  for (int64_t r = 0; r < rows; ++r) {
+    const int32_t g = static_cast<int32_t>(r % G);
+    const int32_t h = static_cast<int32_t>((r / G) % H);
+    const int32_t b = static_cast<int32_t>(r / (static_cast<int64_t>(G) * H));
+    int32_t row_bad = 0;
+    const int32_t ke = ref_top_p_count(mass + r * nK, nK, p, S, &row_bad);
+    int32_t st = ke < 0 ? -1 : 0;
+    if (st == 0) {
+      k_e[r] = ke;
+      st = ref_select_row(mass + r * nK, nK, ke, S - ke, ref_group_uniform(seed, b, h, g), idx + r * S,
+                          log_w + r * S, nullptr, &row_bad);
+    }
+    if (row_bad && bad) {
+#pragma omp atomic write
+      *bad = 1;
+    }
+    status = std::min(status, st);
+  }
+  return status;
+}
+
+// ---------------------------------------------------------------------------
 // [AB] the sparse pass: "the weights become shifts to the sampled attention
 // scores before softmax ... only sampled blocks receive the exact attention
 // computation".  For every query row of the listed groups:
