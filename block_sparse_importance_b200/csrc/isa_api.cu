@@ -158,7 +158,8 @@ isa_status do_score(isa_context* ctx, const isa_shape* s, const void* q, const v
 }
 
 isa_status do_select(isa_context* ctx, const isa_shape* s, const float* mass, int32_t ne, int32_t ns, uint64_t seed,
-                     int32_t* idx, float* log_w, cudaStream_t st, int h_base = 0, int b_base = 0) {
+                     int32_t* idx, float* log_w, cudaStream_t st, int h_base = 0, int b_base = 0,
+                     const int32_t* ne_rows = nullptr) {
   ISA_TRY(check_ptr(ctx, mass, "mass", 4));
   ISA_TRY(check_ptr(ctx, idx, "idx", 4));
   ISA_TRY(check_ptr(ctx, log_w, "log_w", 4));
@@ -179,6 +180,7 @@ isa_status do_select(isa_context* ctx, const isa_shape* s, const float* mass, in
   l.mass = mass;
   l.idx = idx;
   l.log_w = log_w;
+  l.ne_rows = ne_rows;
   l.status = ctx->d_status;
   return cuda_status(ctx, launch_select(l, st), "isa_select");
 }
@@ -373,6 +375,28 @@ isa_status isa_select(isa_context* ctx, const isa_shape* shape, const float* mas
   DeviceGuard g(ctx->device);
   if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
   return do_select(ctx, shape, mass, n_exact, n_sample, seed, idx, log_w, static_cast<cudaStream_t>(stream));
+}
+
+isa_status isa_select_top_p(isa_context* ctx, const isa_shape* shape, const float* mass, double top_p,
+                            int32_t n_select, uint64_t seed, int32_t* idx, float* log_w, int32_t* n_exact_rows,
+                            void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  ISA_TRY(check_ptr(ctx, mass, "mass", 4));
+  ISA_TRY(check_ptr(ctx, idx, "idx", 4));
+  ISA_TRY(check_ptr(ctx, log_w, "log_w", 4));
+  ISA_TRY(check_ptr(ctx, n_exact_rows, "n_exact_rows", 4));
+  if (!(top_p > 0.0) || top_p > 1.0) return fail(ctx, ISA_ERR_INVALID_ARG, "top_p = %g: need 0 < top_p <= 1", top_p);
+  const int nK = nblocks(shape);
+  if (n_select < 1 || n_select > nK)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "n_select = %d: need 1 <= n_select <= nK = %d", n_select, nK);
+  if (nK > 16384) return fail(ctx, ISA_ERR_UNSUPPORTED, "nK = %d key blocks: at most 16384 are built", nK);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int rows = shape->batch * shape->heads * shape->num_groups;
+  ISA_TRY(cuda_status(ctx, launch_top_p_count(mass, rows, nK, top_p, n_select, n_exact_rows, ctx->d_status, st),
+                      "isa_select_top_p"));
+  return do_select(ctx, shape, mass, n_select, 0, seed, idx, log_w, st, 0, 0, n_exact_rows);
 }
 
 size_t isa_attention_workspace_bytes(const isa_shape* s) { return s ? attn_ws_bytes(s) : 0; }

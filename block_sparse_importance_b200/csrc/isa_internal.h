@@ -52,9 +52,15 @@ struct SelectLaunch {
   const float* mass;
   int32_t* idx;
   float* log_w;
+  // per-row exact-set sizes (top-p rule), or NULL for the fixed n_exact; with
+  // it, n_exact + n_sample is the plan size and row r uses ne_rows[r] exact
+  const int32_t* ne_rows;
   int* status;
 };
 int launch_select(const SelectLaunch& s, cudaStream_t stream);
+// Exact-set sizes under the top-p rule, one per plan row, into ne_rows.
+int launch_top_p_count(const float* mass, int rows, int nK, double top_p, int S, int32_t* ne_rows, int* status,
+                       cudaStream_t stream);
 
 // ---------------------------------------------------------------- scorer
 struct ScoreLaunch {

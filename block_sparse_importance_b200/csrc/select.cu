@@ -128,6 +128,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   const int b = static_cast<int>(row / (static_cast<int64_t>(a.G) * a.H));
   const float* m = a.mass + row * nK;
   const int S = a.n_exact + a.n_sample;
+  // the row's split of the plan: fixed, or per row (top-p rule)
+  const int n_exact = a.ne_rows ? min(max(a.ne_rows[row], 0), S) : a.n_exact;
+  const int n_sample = S - n_exact;
   const int E = ((nK + kSelThreads - 1) / kSelThreads) | 1;
   const int i0 = min(nK, tid * E), i1 = min(nK, i0 + E);
 
@@ -147,9 +150,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   __syncthreads();
 
   // ---- exact set: the n_exact largest keys, ties to the lower index
-  if (a.n_exact > 0) {
+  if (n_exact > 0) {
     uint32_t prefix = 0, mask = 0;
-    if (tid == 0) sh.remaining = a.n_exact;
+    if (tid == 0) sh.remaining = n_exact;
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += kSelThreads) sh.hist[i] = 0;
       __syncthreads();
@@ -206,13 +209,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
 
   // ---- weights and capping over the rest (all per-block work is on the
   // thread's own segment; only the totals cross threads)
-  const int n_rest = nK - a.n_exact;
+  const int n_rest = nK - n_exact;
   int n_left = 0;
   uint64_t T = 0;
-  if (a.n_sample >= n_rest) {
+  if (n_sample >= n_rest) {
     for (int i = i0; i < i1; ++i)
       if (!(flag[i] & 1)) flag[i] |= 2;
-  } else if (a.n_sample > 0) {
+  } else if (n_sample > 0) {
     uint32_t kmax = 0;
     for (int i = i0; i < i1; ++i)
       if (!(flag[i] & 1)) kmax = max(kmax, key[i]);
@@ -232,7 +235,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
       for (int i = i0; i < i1; ++i)
         if (!(flag[i] & 3)) t += wq[i];
       T = block_sum_u64(t, sh);
-      n_left = a.n_sample - n_capped;
+      n_left = n_sample - n_capped;
       uint64_t add = 0;
       for (int i = i0; i < i1; ++i)
         if (!(flag[i] & 3) && static_cast<uint64_t>(n_left) * wq[i] >= T) ++add;
@@ -292,11 +295,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   }
   uint64_t tot;
   const uint64_t pre = block_scan_u64((ne << 32) | nr, sh, &tot);  // both counts < 2^32
-  uint64_t pe = pre >> 32, pr = static_cast<uint64_t>(a.n_exact) + (pre & 0xFFFFFFFFull);
+  uint64_t pe = pre >> 32, pr = static_cast<uint64_t>(n_exact) + (pre & 0xFFFFFFFFull);
   for (int i = i0; i < i1; ++i) {
     const uint8_t f = flag[i];
     if (f & 1) {
-      if (pe < static_cast<uint64_t>(a.n_exact)) {
+      if (pe < static_cast<uint64_t>(n_exact)) {
         out_idx[pe] = i;
         out_lw[pe] = 0.0f;
       }
@@ -312,7 +315,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   }
   const uint64_t tot_e = tot >> 32, tot_r = tot & 0xFFFFFFFFull;
   if (tid == 0) {
-    if (sh.bad || tot_e != static_cast<uint64_t>(a.n_exact) || tot_e + tot_r != static_cast<uint64_t>(S))
+    if (sh.bad || tot_e != static_cast<uint64_t>(n_exact) || tot_e + tot_r != static_cast<uint64_t>(S))
       atomicCAS(a.status, 0, kStatusDeviceCheck);
   }
 }
@@ -388,16 +391,19 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
     key[v] = k;  // blocks past the row are 0 and never counted (v >= nv)
   }
   const int S = a.n_exact + a.n_sample;
+  // the row's split of the plan: fixed, or per row (top-p rule)
+  const int n_exact = a.ne_rows ? min(max(a.ne_rows[row], 0), S) : a.n_exact;
+  const int n_sample = S - n_exact;
   // ---- exact set: threshold t = largest key with #{key >= t} >= n_exact
   uint64_t ex = 0;  // bit v: block base+v is exact
-  if (a.n_exact > 0) {
+  if (n_exact > 0) {
     uint32_t t = 0;
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = t | (1u << bit);
       uint32_t c = 0;
 #pragma unroll
       for (int v = 0; v < VPL; ++v) c += (v < nv && key[v] >= cand) ? 1u : 0u;
-      if (__reduce_add_sync(0xffffffffu, c) >= static_cast<uint32_t>(a.n_exact)) t = cand;
+      if (__reduce_add_sync(0xffffffffu, c) >= static_cast<uint32_t>(n_exact)) t = cand;
     }
     uint32_t gt = 0, eq = 0;
 #pragma unroll
@@ -405,7 +411,7 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
       gt += (v < nv && key[v] > t) ? 1u : 0u;
       eq += (v < nv && key[v] == t) ? 1u : 0u;
     }
-    const uint32_t need = static_cast<uint32_t>(a.n_exact) - __reduce_add_sync(0xffffffffu, gt);
+    const uint32_t need = static_cast<uint32_t>(n_exact) - __reduce_add_sync(0xffffffffu, gt);
     uint32_t rank = warp_excl_u32(eq, lane);
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
@@ -417,14 +423,14 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
     }
   }
   // ---- the rest: weights (into the shared slice), capping, systematic PPS
-  const int n_rest = nK - a.n_exact;
+  const int n_rest = nK - n_exact;
   uint64_t cap = 0, drawn = 0;  // bit v: capped (or taken whole), drawn
   uint64_t T = 0;
   int n_left = 0;
-  if (a.n_sample >= n_rest) {
+  if (n_sample >= n_rest) {
     for (int v = 0; v < nv; ++v)
       if (!((ex >> v) & 1)) cap |= 1ull << v;
-  } else if (a.n_sample > 0) {
+  } else if (n_sample > 0) {
     uint32_t kmax = 0;
 #pragma unroll
     for (int v = 0; v < VPL; ++v)
@@ -449,7 +455,7 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
       for (int v = 0; v < nv; ++v)
         if (!((cap >> v) & 1)) tl += st[at(base + v)];
       T = warp_sum_u64(tl);
-      n_left = a.n_sample - n_capped;
+      n_left = n_sample - n_capped;
       uint32_t add = 0;
       uint64_t newcap = 0;
       for (int v = 0; v < nv; ++v) {
@@ -506,12 +512,12 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
   float* out_lw = a.log_w + row * S;
   const uint32_t ne = __popcll(ex), nr = __popcll(cap | drawn);
   uint32_t pe = warp_excl_u32(ne, lane);
-  uint32_t pr = static_cast<uint32_t>(a.n_exact) + warp_excl_u32(nr, lane);
+  uint32_t pr = static_cast<uint32_t>(n_exact) + warp_excl_u32(nr, lane);
   const double lnT = T > 0 ? log(static_cast<double>(T)) : 0.0;
   for (int v = 0; v < nv; ++v) {
     const int i = base + v;
     if ((ex >> v) & 1) {
-      if (pe < static_cast<uint32_t>(a.n_exact)) {
+      if (pe < static_cast<uint32_t>(n_exact)) {
         out_idx[pe] = i;
         out_lw[pe] = 0.0f;
       }
@@ -528,8 +534,90 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
   }
   const uint32_t tot_e = __reduce_add_sync(0xffffffffu, ne), tot_r = __reduce_add_sync(0xffffffffu, nr);
   const bool any_bad = __any_sync(0xffffffffu, bad);
-  if (lane == 0 && (any_bad || tot_e != static_cast<uint32_t>(a.n_exact) || tot_e + tot_r != static_cast<uint32_t>(S)))
+  if (lane == 0 && (any_bad || tot_e != static_cast<uint32_t>(n_exact) || tot_e + tot_r != static_cast<uint32_t>(S)))
     atomicCAS(a.status, 0, kStatusDeviceCheck);
+}
+
+// ---------------------------------------------------------------------------
+// Exact-set size by a share of the mass (the top-p rule of "iCATS": sparsity
+// set by the share p of attention mass kept), one CTA per plan row, thread t
+// over the contiguous blocks [t E, (t+1) E).  In exact integers, as the plan:
+//   q_b = floor(m_b / m_max * 2^31) in fp64 for m_b > 0 (0 otherwise),
+//   target = ceil(p * sum q) in fp64 (the sum is below 2^45: exact),
+//   k_e = min(S, smallest k whose k largest blocks, ties to the lower block,
+//         sum to >= target).
+// The largest key t with sum_{key >= t} q >= target is found bit by bit; all
+// blocks above t are in, and of the blocks at t (equal q) the lowest
+// ceil((target - sum_{key > t} q) / q_t).
+__global__ void __launch_bounds__(kSelThreads) top_p_count_kernel(const float* __restrict__ mass, int nK,
+                                                                  double top_p, int S, int32_t* __restrict__ ne_rows,
+                                                                  int* status) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ SelShared sh;
+  uint32_t* key = reinterpret_cast<uint32_t*>(sm);
+  uint32_t* q = key + nK;
+  const int tid = threadIdx.x;
+  const int64_t row = blockIdx.x;
+  const float* m = mass + row * nK;
+  const int E = ((nK + kSelThreads - 1) / kSelThreads) | 1;
+  const int i0 = min(nK, tid * E), i1 = min(nK, i0 + E);
+  if (tid == 0) sh.bad = 0;
+  __syncthreads();
+  for (int i = tid; i < nK; i += kSelThreads) {
+    const float v = m[i];
+    uint32_t k = 0;
+    if (!isfinite(v)) {
+      sh.bad = 1;
+    } else if (v > 0.0f) {
+      k = __float_as_uint(v);
+    }
+    key[i] = k;
+  }
+  __syncthreads();
+  uint32_t kmax = 0;
+  for (int i = i0; i < i1; ++i) kmax = max(kmax, key[i]);
+  kmax = block_max_u32(kmax, sh);
+  const double mmax = static_cast<double>(__uint_as_float(kmax));
+  auto quant = [&](uint32_t k) -> uint32_t {
+    return (k != 0u && mmax > 0.0)
+               ? static_cast<uint32_t>(floor(static_cast<double>(__uint_as_float(k)) / mmax * 2147483648.0))
+               : 0u;
+  };
+  uint64_t local = 0;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t w = quant(key[i]);
+    q[i] = w;
+    local += w;
+  }
+  const uint64_t total = block_sum_u64(local, sh);
+  const uint64_t target = static_cast<uint64_t>(ceil(top_p * static_cast<double>(total)));
+  int k_e = 0;
+  if (target > 0) {
+    uint32_t t = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = t | (1u << bit);
+      uint64_t s = 0;
+      for (int i = i0; i < i1; ++i) s += key[i] >= cand ? q[i] : 0u;
+      if (block_sum_u64(s, sh) >= target) t = cand;
+    }
+    uint64_t gt_sum = 0, gt_cnt = 0;
+    for (int i = i0; i < i1; ++i) {
+      if (key[i] > t) {
+        gt_sum += q[i];
+        ++gt_cnt;
+      }
+    }
+    gt_sum = block_sum_u64(gt_sum, sh);
+    gt_cnt = block_sum_u64(gt_cnt, sh);
+    const uint64_t q_t = quant(t);
+    const uint64_t need = target - gt_sum;  // > 0: t is the largest key that reaches the target
+    const uint64_t at_t = q_t > 0 ? (need + q_t - 1) / q_t : 0;
+    k_e = static_cast<int>(min(static_cast<uint64_t>(S), gt_cnt + at_t));
+  }
+  if (tid == 0) {
+    ne_rows[row] = k_e;
+    if (sh.bad) atomicCAS(status, 0, kStatusDeviceCheck);
+  }
 }
 
 template <int VPL>
@@ -547,6 +635,18 @@ int launch_select_warp(const SelectLaunch& s, cudaStream_t stream) {
 }
 
 }  // namespace
+
+int launch_top_p_count(const float* mass, int rows, int nK, double top_p, int S, int32_t* ne_rows, int* status,
+                       cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(nK) * 8 + 16;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(top_p_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  top_p_count_kernel<<<static_cast<unsigned>(rows), kSelThreads, smem, stream>>>(mass, nK, top_p, S, ne_rows, status);
+  return static_cast<int>(cudaGetLastError());
+}
 
 int launch_select(const SelectLaunch& s, cudaStream_t stream) {
   if (s.nK <= 32 * 8) return launch_select_warp<8>(s, stream);

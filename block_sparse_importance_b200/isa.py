@@ -67,6 +67,7 @@ def lib():
             L.isa_score_workspace_bytes.restype = _sz
             L.isa_score.argtypes = [_P, S, _P, _P, _i32, _i32, _P, _P, _P, _P, _sz, _P]
             L.isa_select.argtypes = [_P, S, _P, _i32, _i32, _u64, _P, _P, _P]
+            L.isa_select_top_p.argtypes = [_P, S, _P, ctypes.c_double, _i32, _u64, _P, _P, _P, _P]
             L.isa_attention_workspace_bytes.argtypes = [S]
             L.isa_attention_workspace_bytes.restype = _sz
             L.isa_attention.argtypes = [_P, S, _P, _P, _P, _P, _P, _i32, _P, _P, _P, _sz, _P]
@@ -80,7 +81,7 @@ def lib():
             L.isa_debug_set.argtypes = [_P, _i32, _u64]
             L.isa_debug_set.restype = ctypes.c_int
             L.isa_attention_noalloc.argtypes = [_P, S, _P, _P, _P, _P, _P, _i32, _P, _P, _P]
-            for name in ("isa_create", "isa_sync_status", "isa_score", "isa_select", "isa_attention",
+            for name in ("isa_create", "isa_sync_status", "isa_score", "isa_select", "isa_select_top_p", "isa_attention",
                          "isa_dense_attention", "isa_pipeline", "isa_pipeline_host", "isa_attention_noalloc"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
@@ -237,6 +238,24 @@ def select(mass, lay: Layout, n_exact: int, n_sample: int, seed: int, idx=None, 
                           _ptr(idx), _ptr(log_w), _stream(stream))
     ctx.check(st, "isa_select")
     return idx, log_w
+
+
+def select_top_p(mass, lay: Layout, top_p: float, n_select: int, seed: int, idx=None, log_w=None, n_exact=None,
+                 ctx: Optional[Context] = None, stream=None):
+    """isa_select_top_p: plan of n_select blocks per row whose exact part
+    keeps a share top_p of the row's mass; returns (idx, log_w, n_exact)
+    with n_exact [B,H,G] int32 the exact-set size of each row."""
+    ctx = ctx or context(mass.device.index or 0)
+    _dev(mass, torch.float32, "mass")
+    shp = (lay.batch, lay.heads, lay.num_groups, n_select)
+    idx = idx if idx is not None else _empty(shp, torch.int32, mass.device)
+    log_w = log_w if log_w is not None else _empty(shp, torch.float32, mass.device)
+    n_exact = n_exact if n_exact is not None else _empty(shp[:3], torch.int32, mass.device)
+    sh = lay.c()
+    st = lib().isa_select_top_p(ctx.handle, ctypes.byref(sh), _ptr(mass), float(top_p), n_select,
+                                ctypes.c_uint64(seed), _ptr(idx), _ptr(log_w), _ptr(n_exact), _stream(stream))
+    ctx.check(st, "isa_select_top_p")
+    return idx, log_w, n_exact
 
 
 def attention(q, k, v, idx, log_w, lay: Layout, out=None, lse=None, workspace=None,

@@ -167,6 +167,26 @@ ISA_API isa_status isa_select(isa_context* ctx, const isa_shape* shape, const fl
                       float* log_w, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * isa_select_top_p -- a plan of n_select blocks per row whose exact part is
+ * set by a share of the mass instead of a fixed count ("iCATS", top-p
+ * sparsity: keep the blocks that carry a share p of the attention mass).
+ * Per row, in exact integers:
+ *   q_b = floor(m_b / max m * 2^31) (fp64; 0 where m_b <= 0),
+ *   target = ceil(top_p * sum_b q_b) (fp64),
+ *   k_e = min(n_select, the fewest blocks, taken by descending mass with
+ *         ties to the lower block, whose q sum reaches target; 0 if target 0);
+ * then the row is planned as isa_select with n_exact = k_e and
+ * n_sample = n_select - k_e (same uniform, weights and row layout), so every
+ * row holds n_select entries and the rest of the budget is sampled.
+ * mass: [B,H,G,nK] fp32.  idx, log_w: [B,H,G,n_select] (written).
+ * n_exact_rows: [B,H,G] int32 (written: k_e per row).  0 < top_p <= 1,
+ * 1 <= n_select <= nK.  Bit-identical to the CPU oracle for identical mass.
+ * ------------------------------------------------------------------------- */
+ISA_API isa_status isa_select_top_p(isa_context* ctx, const isa_shape* shape, const float* mass,
+                            double top_p, int32_t n_select, uint64_t seed, int32_t* idx,
+                            float* log_w, int32_t* n_exact_rows, void* stream);
+
+/* ---------------------------------------------------------------------------
  * isa_attention -- one sparse flash-attention pass over a plan
  * ("AB-Attention": the weights become shifts of the sampled blocks' scores
  * before the softmax, and only selected blocks receive exact attention; small

@@ -16,7 +16,7 @@ def L():
 
 def test_header_declares_the_boundary():
     names = isa.declared_symbols()
-    for n in ["isa_create", "isa_destroy", "isa_score", "isa_select", "isa_attention",
+    for n in ["isa_create", "isa_destroy", "isa_score", "isa_select", "isa_select_top_p", "isa_attention",
               "isa_dense_attention", "isa_sync_status", "isa_status_string", "isa_score_workspace_bytes",
               "isa_attention_workspace_bytes", "isa_pipeline", "isa_pipeline_host"]:
         assert n in names
