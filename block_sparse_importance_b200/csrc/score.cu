@@ -149,8 +149,29 @@ __global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16
     }
     const int n = r1 - r0;
     const uint16_t* qg = q + (bh * N + r0) * D;
+    // rows [cs, cs + rc) of the group into the warp's buffer (zero past rc),
+    // with the column of ones beside each valid row
+    auto load_chunk = [&](int cs, int rc) {
+      __syncwarp();  // every lane is done with the previous rows
+#pragma unroll 8
+      for (int k2 = 0; k2 < kChunkRows * (D / 8) / 32; ++k2) {
+        const int i = lane + 32 * k2;
+        const int r = i / (D / 8), c16 = i - r * (D / 8);
+        const bool in = r < rc;
+        const uint16_t* src = in ? qg + static_cast<int64_t>(cs + r) * D + c16 * 8 : qg;
+        cp_async16_zfill(xs_base + 2u * (r * XS + c16 * 8), src, in ? 16u : 0u);
+      }
+      for (int r = lane; r < kChunkRows; r += 32)
+        *reinterpret_cast<uint4*>(xs + r * XS + D) = make_uint4(r < rc ? 0x3F80u : 0u, 0u, 0u, 0u);
+      cp_async_wait_all();
+      __syncwarp();
+    };
+    // a group of at most 128 rows is loaded once, before the centroids are
+    // initialised from it
+    const bool one_chunk = n <= kChunkRows;
+    if (one_chunk) load_chunk(0, n);
     // this lane's dimensions of centroids gq (+ 8), initialised at rows
-    // floor(c n / C); all gathers of a lane are in flight together
+    // floor(c n / C)
     float mu[NTC][KSTEPS][4];
 #pragma unroll
     for (int h = 0; h < NTC; ++h) {
@@ -161,13 +182,14 @@ __global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int dim = 16 * ks + 2 * tq + (e & 1) + 8 * (e >> 1);
-          mu[h][ks][e] = r >= 0 ? bf16_to_f(qg[static_cast<int64_t>(r) * D + dim]) : 0.0f;
+          mu[h][ks][e] = r < 0 ? 0.0f
+                         : one_chunk ? bf16_to_f(xs[r * XS + dim])
+                                     : bf16_to_f(qg[static_cast<int64_t>(r) * D + dim]);
         }
     }
     int cnt[NTC];
 #pragma unroll
     for (int h = 0; h < NTC; ++h) cnt[h] = 0;
-    const bool one_chunk = n <= kChunkRows;
     for (int it = 0; it < iters; ++it) {
       // centroids as bf16 hi + lo B fragments, and |mu_c|^2
       uint32_t bhi[NTC][KSTEPS][2], blo[NTC][KSTEPS][2];
@@ -204,21 +226,7 @@ __global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16
         for (int k = 0; k < 4; ++k) sums[i][k] = 0.0f;
       for (int cs = 0; cs < n; cs += kChunkRows) {
         const int rc = min(kChunkRows, n - cs);
-        if (!(one_chunk && it > 0)) {
-          __syncwarp();  // every lane is done with the previous rows
-#pragma unroll 8
-          for (int k2 = 0; k2 < kChunkRows * (D / 8) / 32; ++k2) {
-            const int i = lane + 32 * k2;
-            const int r = i / (D / 8), c16 = i - r * (D / 8);
-            const bool in = r < rc;
-            const uint16_t* src = in ? qg + static_cast<int64_t>(cs + r) * D + c16 * 8 : qg;
-            cp_async16_zfill(xs_base + 2u * (r * XS + c16 * 8), src, in ? 16u : 0u);
-          }
-          for (int r = lane; r < kChunkRows; r += 32)
-            *reinterpret_cast<uint4*>(xs + r * XS + D) = make_uint4(r < rc ? 0x3F80u : 0u, 0u, 0u, 0u);
-          cp_async_wait_all();
-          __syncwarp();
-        }
+        if (!one_chunk) load_chunk(cs, rc);
         // assignment: dist_c = |mu_c|^2 - 2 x.mu_c; argmin over c (ties to the
         // lower c) of rows gq and gq + 8 of row tile rt
         auto pick = [&](int rt, const float (&acc)[NTC][4]) {
@@ -251,29 +259,39 @@ __global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16
           }
         };
         const int nrt = (rc + 15) / 16;  // row tiles holding rows of the group
-        {
-          for (int rt = 0; rt < kChunkRows / 16; ++rt) {
-            if (rt >= nrt) {
-              if (lane < 16) assign[16 * rt + lane] = -1;
-              continue;
-            }
-            float acc[NTC][4];
+        // four row tiles at a time, so that four independent product chains
+        // are in flight (rows past rc are zero and get assignment -1)
+        constexpr int kRt = 4;
+        for (int rt0 = 0; rt0 < kChunkRows / 16; rt0 += kRt) {
+          if (rt0 >= nrt) {
+            if (lane < 16 * kRt / 2) reinterpret_cast<int2*>(assign + 16 * rt0)[lane] = make_int2(-1, -1);
+            continue;
+          }
+          float acc[kRt][NTC][4];
+#pragma unroll
+          for (int t = 0; t < kRt; ++t)
 #pragma unroll
             for (int i = 0; i < NTC; ++i)
 #pragma unroll
-              for (int k = 0; k < 4; ++k) acc[i][k] = 0.0f;
+              for (int k = 0; k < 4; ++k) acc[t][i][k] = 0.0f;
 #pragma unroll
-            for (int ks = 0; ks < KSTEPS; ++ks) {
-              uint32_t a[4];
-              ldsm_x4(a, xs_base + 2u * ((16 * rt + a_row) * XS + ks * 16 + a_col));
+          for (int ks = 0; ks < KSTEPS; ++ks) {
+            uint32_t a[kRt][4];
 #pragma unroll
-              for (int nt = 0; nt < NTC; ++nt) {
-                mma_16816(acc[nt], a, bhi[nt][ks][0], bhi[nt][ks][1]);
-                mma_16816(acc[nt], a, blo[nt][ks][0], blo[nt][ks][1]);
-              }
-            }
-            pick(rt, acc);
+            for (int t = 0; t < kRt; ++t)
+              ldsm_x4(a[t], xs_base + 2u * ((16 * (rt0 + t) + a_row) * XS + ks * 16 + a_col));
+            // the hi and lo products of one accumulator are kRt * NTC issues apart
+#pragma unroll
+            for (int t = 0; t < kRt; ++t)
+#pragma unroll
+              for (int nt = 0; nt < NTC; ++nt) mma_16816(acc[t][nt], a[t], bhi[nt][ks][0], bhi[nt][ks][1]);
+#pragma unroll
+            for (int t = 0; t < kRt; ++t)
+#pragma unroll
+              for (int nt = 0; nt < NTC; ++nt) mma_16816(acc[t][nt], a[t], blo[nt][ks][0], blo[nt][ks][1]);
           }
+#pragma unroll
+          for (int t = 0; t < kRt; ++t) pick(rt0 + t, acc[t]);
         }
         __syncwarp();
         // cluster sums (and counts, from the column of ones): one-hot^T x
@@ -345,11 +363,14 @@ __global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16
 //           tcgen05.mma products (hi.hi + hi.lo + lo.hi) accumulate in TMEM;
 //   pass 0  each row's online max and sum of exp over all key blocks;
 //   pass 1  the logits again, p = n_c exp(l - max) / sum, summed over the Cp
-//           rows of each group by a reduce-scatter across lanes, and written.
-// Warps 0-3: one thread per centroid row (TMEM lane); warp 4: TMA producer of
-// the kbar tiles (128 blocks x d, hi and lo) into a 2-stage ring; warp 5:
-// MMA issue.  S is double-buffered in TMEM (2 x 128 columns).
-constexpr int kMassThreads = 192;
+//           rows of each group through a shared-memory transpose, and written.
+// Warps 0-7: softmax, two warps per centroid row quarter (TMEM lanes
+// 32 (w & 3) ..), warp w taking columns 64 (w >> 2) .. + 63 of every tile;
+// warp 8: TMA producer of the kbar tiles (128 blocks x d, hi and lo) into a
+// 2-stage ring; warp 9: MMA issue.  S is double-buffered in TMEM (2 x 128
+// columns).
+constexpr int kMassSoftmaxWarps = 8;
+constexpr int kMassThreads = (kMassSoftmaxWarps + 2) * 32;
 constexpr int kMassRing = 2;
 
 template <int D>
@@ -360,9 +381,12 @@ struct MassLayout {
   static constexpr uint32_t kStage = 2 * kTile;            // kbar hi + lo
   static constexpr uint32_t kBar = kRing + kMassRing * kStage;
   static constexpr int kBarFull = 0, kBarEmpty = kMassRing, kBarSFull = 2 * kMassRing, kBarSFree = kBarSFull + 2,
-                       kBarFinal = kBarSFree + 2, kNumBars = kBarFinal + 1;
+                       kBarFinal = kBarSFree + 2, kBarXchg = kBarFinal + 1, kNumBars = kBarXchg + 1;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;
-  static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
+  static constexpr uint32_t kXchg = (kMisc + 16 + 15) & ~15u;  // [2 halves][128 rows] (max, sum)
+  static constexpr int kXS = 20;  // row stride (floats) of the transpose buffers: 16 columns + 4
+  static constexpr uint32_t kXpose = kXchg + 2 * 128 * 8;
+  static constexpr uint32_t kAlloc = kXpose + kMassSoftmaxWarps * 32 * kXS * 4 + 1024;
 };
 
 template <int D, int Cp>
@@ -373,6 +397,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
   using namespace isa_dev;
   using L = MassLayout<D>;
   constexpr int kGroupsPerTile = 128 / Cp;
+  constexpr int kProducer = kMassSoftmaxWarps, kMma = kMassSoftmaxWarps + 1;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -421,13 +446,14 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::kBarSFull + i), 1);
-      mbar_init(bar(L::kBarSFree + i), 128);
+      mbar_init(bar(L::kBarSFree + i), kMassSoftmaxWarps * 32);
     }
     mbar_init(bar(L::kBarFinal), 1);
+    mbar_init(bar(L::kBarXchg), kMassSoftmaxWarps * 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMma) {
     tmem_alloc(smem_addr(tmem_slot), 256);
     tmem_relinquish();
   }
@@ -438,7 +464,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kProducer) {
     // ------------------------------------------------------------ producer
     uint32_t issued = 0;
     bool ok = true;
@@ -469,7 +495,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMma) {
     // ----------------------------------------------------------------- MMA
     // The whole warp runs the loop and waits; one elected lane issues.  The
     // shared-memory descriptors are built once and advanced by adds to their
@@ -506,95 +532,161 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     }
   } else {
     // ------------------------------------------------------------- softmax
-    const int row = tid;  // centroid row == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // Thread = centroid row = TMEM lane; the two warps of a row quarter take
+    // the two 64-column halves of every tile.  With s = scale log2(e) > 0
+    // the log2-domain logit of block b is z_b = s x_b for the raw product
+    // x_b (a partial tail block adds log2(L_b / Bk) to it, folded into x as
+    // an offset; columns past nK become -inf), so the running max is taken
+    // on x.  A half tile comes out of TMEM in one go and the S buffer is
+    // released before any arithmetic.
+    //   pass 0  m = max z and Z = sum 2^(z - m), online over the tiles; the
+    //           two halves' (m, Z) are merged once through shared memory;
+    //   pass 1  n_c 2^(z - m) / Z = 2^(s x - o) with o = m - log2(n_c / Z):
+    //           one paired FMA and one ex2 per value; the Cp rows of each
+    //           group are summed through a per-warp shared-memory transpose
+    //           of 16 columns at a time (row stride 20 floats: the row
+    //           writes are free of bank conflicts).
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;  // centroid row == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 64;
     const int gl = row / Cp, c = row - gl * Cp, g = g0 + gl;
     const float n_c = (c < C && g < G) ? static_cast<float>(counts[(bh * G + g) * C + c]) : 0.0f;
     const int tail_rows = N - (nK - 1) * Bk;
-    const float tail_adj = tail_rows < Bk ? log2f(static_cast<float>(tail_rows) / static_cast<float>(Bk)) : 0.0f;
-    float m_run = -INFINITY, z_run = 0.0f, w = 0.0f;
-    constexpr int kCols = 32 / Cp;  // columns a lane owns after the reduce-scatter of a 32-column chunk
+    const float tail_dx =
+        tail_rows < Bk ? log2f(static_cast<float>(tail_rows) / static_cast<float>(Bk)) / scale_log2 : 0.0f;
+    constexpr int kCols = 16 / Cp > 0 ? 16 / Cp : 1;  // columns a lane sums and stores per 16-column chunk
+    float* xp = reinterpret_cast<float*>(smem + L::kXpose) + warp * 32 * L::kXS;
+    float2* xchg = reinterpret_cast<float2*>(smem + L::kXchg);
+    const int p = lane & (Cp - 1), gw = lane / Cp;  // this lane's slice and group within the warp
+    const uint64_t ss = f2_pack(scale_log2, scale_log2);
+    float m_run = -INFINITY, z_run = 0.0f, o = INFINITY;
     for (int i = 0; i < n_items; ++i) {
       const int pass = i / T, j = i - pass * T;
       const uint32_t buf = i & 1;
       if (!mbar_wait(bar(L::kBarSFull + buf), (i >> 1) & 1u, abort_flag, kWaitTimeoutNs)) break;
       tc_fence_after();
-      const int col0 = j * 128;
+      uint32_t sv[2][32];
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) tmem_ld32(lane_base + buf * 128 + 32 * cc, sv[cc]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarSFree + buf));
+      const int col0 = j * 128 + half * 64;
+      if (j == T - 1) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int b = col0 + 32 * cc + e;
+            float xv = __uint_as_float(sv[cc][e]);
+            if (b == nK - 1) xv += tail_dx;
+            sv[cc][e] = __float_as_uint(b < nK ? xv : -INFINITY);
+          }
+      }
       if (pass == 0) {
-        float tmax = -INFINITY;
-        float zs[4][32];
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t sv[32];
-          tmem_ld32(lane_base + buf * 128 + 32 * cc, sv);
-          tmem_wait_ld();
+        for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int b = col0 + 32 * cc + e;
-            float z = __uint_as_float(sv[e]) * scale_log2;
-            if (b == nK - 1) z += tail_adj;
-            z = b < nK ? z : -INFINITY;
-            zs[cc][e] = z;
-            tmax = fmaxf(tmax, z);
-          }
+          for (int e = 0; e < 32; e += 8)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mx[k] = fmax3f(mx[k], __uint_as_float(sv[cc][e + k]), __uint_as_float(sv[cc][e + 4 + k]));
+        const float xm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        const float m_new = fmaxf(m_run, xm * scale_log2);
+        // a half tile past nK is all -inf: nothing to add
+        if (m_new != -INFINITY) {
+          const uint64_t nm = f2_pack(-m_new, -m_new);
+          uint64_t part[4] = {0ull, 0ull, 0ull, 0ull};  // +0.0f pairs
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float y0, y1;
+              f2_unpack(fma_f32x2(f2_pack(__uint_as_float(sv[cc][e]), __uint_as_float(sv[cc][e + 1])), ss, nm), y0,
+                        y1);
+              part[(e >> 1) & 3] = add_f32x2(part[(e >> 1) & 3], f2_pack(fast_exp2(y0), fast_exp2(y1)));
+            }
+          const uint64_t p01 = add_f32x2(add_f32x2(part[0], part[1]), add_f32x2(part[2], part[3]));
+          float s0, s1;
+          f2_unpack(p01, s0, s1);
+          z_run = (m_run == -INFINITY ? 0.0f : z_run * fast_exp2(m_run - m_new)) + (s0 + s1);
+          m_run = m_new;
         }
-        const float m_new = fmaxf(m_run, tmax);
-        float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) part[e & 3] += fast_exp2(zs[cc][e] - m_new);
-        z_run = (m_run == -INFINITY ? 0.0f : z_run * fast_exp2(m_run - m_new)) + ((part[0] + part[1]) + (part[2] + part[3]));
-        m_run = m_new;
-        if (j == T - 1) w = z_run > 0.0f ? n_c / z_run : 0.0f;
+        if (j == T - 1) {
+          // merge the two halves' (m, Z) in a fixed order, so that both warps
+          // of the row get the same o
+          xchg[half * 128 + row] = make_float2(m_run, z_run);
+          mbar_arrive(bar(L::kBarXchg));
+          if (!mbar_wait(bar(L::kBarXchg), 0, abort_flag, kWaitTimeoutNs)) break;
+          const float2 h0 = xchg[row], h1 = xchg[128 + row];
+          const float m = fmaxf(h0.x, h1.x);
+          const float z = (h0.x == -INFINITY ? 0.0f : h0.y * fast_exp2(h0.x - m)) +
+                          (h1.x == -INFINITY ? 0.0f : h1.y * fast_exp2(h1.x - m));
+          const float w = z > 0.0f ? n_c / z : 0.0f;
+          o = w > 0.0f ? m - log2f(w) : INFINITY;
+        }
       } else {
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t sv[32];
-          tmem_ld32(lane_base + buf * 128 + 32 * cc, sv);
-          tmem_wait_ld();
-          float v[32];
+        const uint64_t no = f2_pack(-o, -o);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int b = col0 + 32 * cc + e;
-            float z = __uint_as_float(sv[e]) * scale_log2;
-            if (b == nK - 1) z += tail_adj;
-            v[e] = b < nK ? w * fast_exp2(z - m_run) : 0.0f;
+        for (int ch = 0; ch < 4; ++ch) {
+          const int cc = ch >> 1, e0 = (ch & 1) * 16;
+          float v[16];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float y0, y1;
+            f2_unpack(fma_f32x2(f2_pack(__uint_as_float(sv[cc][e0 + e]), __uint_as_float(sv[cc][e0 + e + 1])), ss,
+                                no),
+                      y0, y1);
+            v[e] = fast_exp2(y0);
+            v[e + 1] = fast_exp2(y1);
           }
-          // reduce-scatter over the Cp rows of each group: lane p of a group
-          // ends with the group's sums for columns [p * kCols, (p+1) * kCols)
+          __syncwarp();  // every lane has read the previous chunk
 #pragma unroll
-          for (int m = Cp / 2, cnt = 16; m >= 1; m >>= 1, cnt >>= 1) {
-            const bool up = (lane & m) != 0;
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<float4*>(xp + lane * L::kXS + 4 * k) =
+                make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          __syncwarp();
+          float acc[kCols];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              if (e < cnt) {
-                const float mine = up ? v[cnt + e] : v[e];
-                const float other = up ? v[e] : v[cnt + e];
-                v[e] = mine + __shfl_xor_sync(0xffffffffu, other, m);
+          for (int e = 0; e < kCols; ++e) acc[e] = 0.0f;
+#pragma unroll
+          for (int r = 0; r < Cp; ++r) {
+            const float* src = xp + (gw * Cp + r) * L::kXS + p * kCols;
+            if constexpr (kCols % 4 == 0) {
+#pragma unroll
+              for (int e = 0; e < kCols; e += 4) {
+                const float4 t = *reinterpret_cast<const float4*>(src + e);
+                acc[e] += t.x;
+                acc[e + 1] += t.y;
+                acc[e + 2] += t.z;
+                acc[e + 3] += t.w;
               }
+            } else if constexpr (kCols == 2) {
+              const float2 t = *reinterpret_cast<const float2*>(src);
+              acc[0] += t.x;
+              acc[1] += t.y;
+            } else {
+#pragma unroll
+              for (int e = 0; e < kCols; ++e) acc[e] += src[e];
             }
           }
-          const int p = lane & (Cp - 1);
           if (g < G) {
             float* dst = mass + (bh * G + g) * nK;
 #pragma unroll
             for (int e = 0; e < kCols; ++e) {
-              const int b = col0 + 32 * cc + p * kCols + e;
-              if (b < nK) dst[b] = v[e];
+              const int b = col0 + 16 * ch + p * kCols + e;
+              if (b < nK) dst[b] = acc[e];
             }
           }
         }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(L::kBarSFree + buf));
     }
   }
   tc_fence_before();
   __syncthreads();
   if (tid == 0 && *abort_flag) atomicCAS(status, 0, kStatusTimeout);
-  if (warp == 5) {
+  if (warp == kMma) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 256);
