@@ -66,6 +66,13 @@ def _load():
             lib.ref_attention.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, i32, P, P, i32, f64,
                                           P, i32, P, P, i32]
             lib.ref_dense_attention.argtypes = [P, P, P, i32, i32, f64, P, i32, P, P, i32]
+            lib.ref_cluster_assign.argtypes = [P, i32, i32, P, i32, f64, P, P]
+            lib.ref_cluster_assign.restype = None
+            lib.ref_cluster_sort.argtypes = [P, i32, i32, P, P]
+            lib.ref_cluster_sort.restype = None
+            lib.ref_cluster_update.argtypes = [P, i32, i32, P, i32, P, P]
+            lib.ref_cluster_update.restype = None
+            lib.ref_cluster_tokens.argtypes = [P, i32, i32, i32, i32, i32, f64, P, P, P, P, P, i32]
             lib.ref_num_threads.restype = i32
             _lib = lib
     return _lib
@@ -116,6 +123,63 @@ def kmeans_group(q_rows: np.ndarray, n_clusters: int, n_iters: int, tie_rel: flo
     cnt = np.zeros(n_clusters, np.int32)
     amb = _load().ref_kmeans_group(_p(q_rows), n, d, n_clusters, n_iters, tie_rel, _p(mu), _p(cnt))
     return mu, cnt, bool(amb)
+
+
+def cluster_assign(x_rows: np.ndarray, mu: np.ndarray, tie_rel: float = KMEANS_TIE_REL):
+    """One assignment round: x_rows [n, d] uint16 bf16 bits, mu [C, d] ->
+    (labels [n] i32, ambiguous [n] bool)."""
+    x_rows = _c(x_rows, np.uint16)
+    mu = _c(mu, np.float64)
+    n, d = x_rows.shape
+    C = mu.shape[0]
+    lab = np.zeros(n, np.int32)
+    amb = np.zeros(n, np.int32)
+    _load().ref_cluster_assign(_p(x_rows), n, d, _p(mu), C, tie_rel, _p(lab), _p(amb))
+    return lab, amb.astype(bool)
+
+
+def cluster_sort(labels: np.ndarray, n_clusters: int):
+    """Stable counting sort: labels [n] -> (perm [n] i32, offsets [C + 1] i32)."""
+    labels = _c(labels, np.int32)
+    if labels.size and (labels.min() < 0 or labels.max() >= n_clusters):
+        raise ValueError("labels out of range")
+    perm = np.zeros(labels.size, np.int32)
+    off = np.zeros(n_clusters + 1, np.int32)
+    _load().ref_cluster_sort(_p(labels), labels.size, n_clusters, _p(perm), _p(off))
+    return perm, off
+
+
+def cluster_update(x_rows: np.ndarray, labels: np.ndarray, mu: np.ndarray):
+    """Mean update: returns (new mu [C, d] f64, counts [C] i32); an empty
+    cluster keeps its row of `mu`."""
+    x_rows = _c(x_rows, np.uint16)
+    labels = _c(labels, np.int32)
+    mu = np.array(mu, dtype=np.float64, copy=True, order="C")
+    n, d = x_rows.shape
+    C = mu.shape[0]
+    cnt = np.zeros(C, np.int32)
+    _load().ref_cluster_update(_p(x_rows), n, d, _p(labels), C, _p(mu), _p(cnt))
+    return mu, cnt
+
+
+def cluster_tokens(x: np.ndarray, n_clusters: int, n_iters: int, tie_rel: float = KMEANS_TIE_REL,
+                   threads: int = 0):
+    """Clustering of every (batch, head) over the whole sequence.
+    x: [B, H, N, d] uint16 bf16 bits -> (labels [B,H,N], perm [B,H,N],
+    offsets [B,H,C+1], mu [B,H,C,d] f64, ambiguous [B,H] bool)."""
+    x = _c(x, np.uint16)
+    B, H, N, d = x.shape
+    C = n_clusters
+    lab = np.zeros((B, H, N), np.int32)
+    perm = np.zeros((B, H, N), np.int32)
+    off = np.zeros((B, H, C + 1), np.int32)
+    mu = np.zeros((B, H, C, d), np.float64)
+    amb = np.zeros((B, H), np.int32)
+    st = _load().ref_cluster_tokens(_p(x), B * H, N, d, C, n_iters, tie_rel, _p(lab), _p(perm), _p(off), _p(mu),
+                                    _p(amb), threads)
+    if st != 0:
+        raise ValueError("ref_cluster_tokens: need N >= 1, 1 <= C <= N, n_iters >= 1")
+    return lab, perm, off, mu, amb.astype(bool)
 
 
 def mass_group(mu: np.ndarray, counts: np.ndarray, kbar: np.ndarray, L: np.ndarray, scale: float):

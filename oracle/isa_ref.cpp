@@ -24,9 +24,13 @@
 // inclusion probabilities and exact unbiasedness of the weighted numerator
 // and denominator by integration over the uniform; the pages' worked example
 // (pi = 1/4 counts four times); the dense limit against a library attention.
+// Token clustering (the permuted layout): brute-force nearest centroid, the
+// stable sort against a library stable argsort, the mean update against
+// numpy, the one-cluster closed form, a non-increasing objective, and the
+// recovery of well-separated generated clusters.
 // Parity unpinned (fixed by reading, checked only GPU-vs-oracle): the
 // k-means initialisation, the ln(L_b) term of the mass, tie-breaks, canonical
-// plan order, the 2^31 weight quantisation.
+// plan order, the 2^31 weight quantisation, the clustering's round count.
 
 #include <algorithm>
 #include <cmath>
@@ -604,6 +608,118 @@ void ref_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v
     for (int32_t j = 0; j < d; ++j) out[static_cast<int64_t>(i) * d + j] = acc[j] / sum;
     if (lse) lse[i] = mx + std::log(sum);
   }
+}
+
+// ---------------------------------------------------------------------------
+// [IG] / [AB] the permuted layout of permuted block-sparse attention: tokens
+// of one (batch, head) are clustered over the whole sequence ("semantic-
+// aware permutation", the SVG2 layout InstaGen is parameterised by) and
+// reordered so that each cluster's rows are contiguous; a query cluster is
+// then one query group and the reordered keys form the key blocks.
+// (reading) Lloyd's k-means over the N rows of x with C clusters,
+// centroids initialised at rows floor(c N / C), `iters` rounds of
+//   assign  label_r = argmin_c ||x_r - mu_c||^2 (ties to the lower c),
+//   sort    perm = the rows ordered by (label, row): a stable counting sort;
+//           offsets[c] = number of rows with a label below c,
+//   update  mu_c = mean of the rows of cluster c (an empty cluster keeps its
+//           centroid),
+// and the labels, permutation and offsets of the last round are the result.
+// ---------------------------------------------------------------------------
+
+// One assignment round.  x: [n, d] bf16 bits, mu: [C, d].  labels: [n].
+// ambiguous (optional, [n]): 1 where the best and second-best squared
+// distances differ by at most tie_rel * (||x||^2 + ||mu||^2), the margin
+// below which a single-precision implementation may choose differently.
+void ref_cluster_assign(const uint16_t* x, int32_t n, int32_t d, const double* mu, int32_t C, double tie_rel,
+                        int32_t* labels, int32_t* ambiguous) {
+  for (int32_t r = 0; r < n; ++r) {
+    std::vector<double> xr(d);
+    double xx = 0.0;
+    for (int32_t j = 0; j < d; ++j) {
+      xr[j] = bf16_value(x[static_cast<int64_t>(r) * d + j]);
+      xx += xr[j] * xr[j];
+    }
+    double best = INFINITY, second = INFINITY, mm_best = 0.0, mm_second = 0.0;
+    int32_t arg = 0;
+    for (int32_t c = 0; c < C; ++c) {
+      double dist = 0.0, mm = 0.0;
+      for (int32_t j = 0; j < d; ++j) {
+        const double m = mu[static_cast<int64_t>(c) * d + j];
+        dist += (xr[j] - m) * (xr[j] - m);
+        mm += m * m;
+      }
+      if (dist < best) {
+        second = best;
+        mm_second = mm_best;
+        best = dist;
+        mm_best = mm;
+        arg = c;
+      } else if (dist < second) {
+        second = dist;
+        mm_second = mm;
+      }
+    }
+    labels[r] = arg;
+    if (ambiguous) ambiguous[r] = (C > 1 && second - best <= tie_rel * (xx + std::max(mm_best, mm_second))) ? 1 : 0;
+  }
+}
+
+// Stable counting sort of the labels: perm[i] = the i-th row in (label, row)
+// order; offsets: [C + 1], offsets[c] .. offsets[c + 1] the rows of cluster c.
+void ref_cluster_sort(const int32_t* labels, int32_t n, int32_t C, int32_t* perm, int32_t* offsets) {
+  std::vector<int32_t> next(C + 1, 0);
+  for (int32_t r = 0; r < n; ++r) next[labels[r] + 1] += 1;
+  for (int32_t c = 0; c < C; ++c) next[c + 1] += next[c];
+  for (int32_t c = 0; c <= C; ++c) offsets[c] = next[c];
+  for (int32_t r = 0; r < n; ++r) perm[next[labels[r]]++] = r;
+}
+
+// Centroid update from the labels: mu_c = mean of its rows; counts: [C].
+void ref_cluster_update(const uint16_t* x, int32_t n, int32_t d, const int32_t* labels, int32_t C, double* mu,
+                        int32_t* counts) {
+  std::vector<double> sum(static_cast<size_t>(C) * d, 0.0);
+  for (int32_t c = 0; c < C; ++c) counts[c] = 0;
+  for (int32_t r = 0; r < n; ++r) {
+    counts[labels[r]] += 1;
+    for (int32_t j = 0; j < d; ++j)
+      sum[static_cast<int64_t>(labels[r]) * d + j] += bf16_value(x[static_cast<int64_t>(r) * d + j]);
+  }
+  for (int32_t c = 0; c < C; ++c) {
+    if (counts[c] == 0) continue;
+    for (int32_t j = 0; j < d; ++j) mu[static_cast<int64_t>(c) * d + j] = sum[static_cast<int64_t>(c) * d + j] / counts[c];
+  }
+}
+
+// The whole clustering of every (batch, head): x [BH, N, d] bf16 bits.
+// labels, perm: [BH, N]; offsets: [BH, C + 1]; mu: [BH, C, d];
+// ambiguous: [BH] (1 if any round of that head met a near tie).
+int32_t ref_cluster_tokens(const uint16_t* x, int32_t BH, int32_t N, int32_t d, int32_t C, int32_t iters,
+                           double tie_rel, int32_t* labels, int32_t* perm, int32_t* offsets, double* mu,
+                           int32_t* ambiguous, int32_t nthreads) {
+  if (BH < 1 || N < 1 || d < 1 || C < 1 || C > N || iters < 1) return -1;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel for schedule(dynamic)
+  for (int32_t bh = 0; bh < BH; ++bh) {
+    const uint16_t* xb = x + static_cast<int64_t>(bh) * N * d;
+    double* mub = mu + static_cast<int64_t>(bh) * C * d;
+    int32_t* lab = labels + static_cast<int64_t>(bh) * N;
+    for (int32_t c = 0; c < C; ++c) {
+      const int64_t r = (static_cast<int64_t>(c) * N) / C;
+      for (int32_t j = 0; j < d; ++j) mub[static_cast<int64_t>(c) * d + j] = bf16_value(xb[r * d + j]);
+    }
+    std::vector<int32_t> amb(N), counts(C);
+    int32_t any = 0;
+    for (int32_t it = 0; it < iters; ++it) {
+      ref_cluster_assign(xb, N, d, mub, C, tie_rel, lab, amb.data());
+      for (int32_t r = 0; r < N; ++r) any |= amb[r];
+      ref_cluster_update(xb, N, d, lab, C, mub, counts.data());
+    }
+    ref_cluster_sort(lab, N, C, perm + static_cast<int64_t>(bh) * N, offsets + static_cast<int64_t>(bh) * (C + 1));
+    ambiguous[bh] = any;
+  }
+  return 0;
 }
 
 int32_t ref_num_threads(void) {
