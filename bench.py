@@ -249,6 +249,9 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cluster", type=int, default=0,
+                    help="also time the permuted layout's build: isa_cluster of Q and of K with this many clusters "
+                         "(3 rounds) and the row permutations of Q, K and V")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -369,6 +372,38 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         dense_ms = e0.elapsed_time(e1) / 2
+
+    # the permuted layout's build (token clustering of Q and K, then the row
+    # permutations): algorithmic FLOPs are the distance products, 2 N C d per
+    # assignment round per tensor and head
+    if rank == 0 and args.cluster:
+        C_t, it_t = args.cluster, 3
+        cws = torch.empty(isa.cluster_workspace_bytes(q, C_t) + 256, dtype=torch.uint8, device=dev)
+        qp, kp, vp = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def layout_build():
+            rq = isa.cluster(q, C_t, it_t, workspace=cws, ctx=ctx)
+            rk = isa.cluster(k, C_t, it_t, workspace=cws, ctx=ctx)
+            isa.permute_rows(q, rq["perm"], out=qp, ctx=ctx)
+            isa.permute_rows(k, rk["perm"], out=kp, ctx=ctx)
+            isa.permute_rows(v, rk["perm"], out=vp, ctx=ctx)
+
+        layout_build()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(2):
+            layout_build()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        st = ctx.sync_status()
+        if st != isa.ISA_OK:
+            raise RuntimeError("device status after the layout build: %s" % isa.status_string(st))
+        c_ms = e0.elapsed_time(e1) / 2
+        c_flops = 2.0 * N * C_t * d * 2 * B * H * it_t
+        stages["cluster"] = {"ms": c_ms, "n_clusters": C_t, "rounds": it_t, "tflop": c_flops / 1e12,
+                             "tflops": c_flops / (c_ms * 1e-3) / 1e12,
+                             "what": "isa_cluster of Q and of K, then permute_rows of Q, K and V"}
+        del qp, kp, vp, cws
 
     # end to end through the C ABI from pinned host buffers
     e2e = None

@@ -110,6 +110,55 @@ isa_status cuda_status(isa_context* ctx, int e, const char* what) {
     if (s_ != ISA_OK) return s_;    \
   } while (0)
 
+// Shapes of the token-clustering calls: only batch, heads, seq_len and
+// head_dim are read.
+isa_status check_rows_shape(isa_context* ctx, const isa_shape* s) {
+  if (!ctx) return ISA_ERR_INVALID_ARG;
+  ctx->last_error[0] = 0;
+  if (!s) return fail(ctx, ISA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->batch < 1 || s->heads < 1 || s->seq_len < 1)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "batch, heads and seq_len must be >= 1");
+  if (s->head_dim != 64 && s->head_dim != 128)
+    return fail(ctx, ISA_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are built", s->head_dim);
+  const long long bh = static_cast<long long>(s->batch) * s->heads;
+  if (bh * s->seq_len > (1LL << 31) - 1 || bh > 65535)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "tensor too large for the clustering calls");
+  return ISA_OK;
+}
+
+constexpr int kMaxClusters = 8192;
+
+isa_status check_clusters(isa_context* ctx, const isa_shape* s, int32_t C) {
+  if (C < 1 || C > s->seq_len || C > kMaxClusters)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "n_clusters = %d: need 1 <= n_clusters <= min(seq_len, %d)", C, kMaxClusters);
+  return ISA_OK;
+}
+
+size_t cluster_ws(const isa_shape* s, int32_t C) {
+  const size_t BH = static_cast<size_t>(s->batch) * s->heads;
+  const size_t cp = static_cast<size_t>(cluster_cpad(C));
+  return 2 * round_up(BH * cp * s->head_dim * 2) + round_up(BH * cp * 4);
+}
+
+ClusterLaunch cluster_launch(const isa_shape* s, int32_t C, const void* x, float* mu, void* ws) {
+  ClusterLaunch l{};
+  l.BH = s->batch * s->heads;
+  l.N = s->seq_len;
+  l.D = s->head_dim;
+  l.C = C;
+  l.Cpad = cluster_cpad(C);
+  l.x = x;
+  l.mu = mu;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const size_t BH = static_cast<size_t>(l.BH);
+  l.mu_hi = reinterpret_cast<uint16_t*>(w);
+  w += round_up(BH * l.Cpad * l.D * 2);
+  l.mu_lo = reinterpret_cast<uint16_t*>(w);
+  w += round_up(BH * l.Cpad * l.D * 2);
+  l.mu_nsq = reinterpret_cast<float*>(w);
+  return l;
+}
+
 size_t attn_ws_bytes(const isa_shape* s) {
   const bool list = s->q_offsets != nullptr || s->q_block > 128;
   return list ? round_up(attn_list_workspace_bytes(s->seq_len, s->num_groups)) : 0;
@@ -397,6 +446,136 @@ isa_status isa_select_top_p(isa_context* ctx, const isa_shape* shape, const floa
   ISA_TRY(cuda_status(ctx, launch_top_p_count(mass, rows, nK, top_p, n_select, n_exact_rows, ctx->d_status, st),
                       "isa_select_top_p"));
   return do_select(ctx, shape, mass, n_select, 0, seed, idx, log_w, st, 0, 0, n_exact_rows);
+}
+
+size_t isa_cluster_workspace_bytes(const isa_shape* shape, int32_t n_clusters) {
+  if (!shape || n_clusters < 1 || n_clusters > kMaxClusters || shape->batch < 1 || shape->heads < 1 ||
+      shape->head_dim < 1)
+    return 0;
+  return cluster_ws(shape, n_clusters);
+}
+
+isa_status isa_cluster(isa_context* ctx, const isa_shape* shape, const void* x, int32_t n_clusters, int32_t n_iters,
+                       float* centroids, int32_t* labels, int32_t* perm, int32_t* offsets, int32_t* groups,
+                       int32_t* n_groups, void* workspace, size_t workspace_bytes, void* stream) {
+  ISA_TRY(check_rows_shape(ctx, shape));
+  ISA_TRY(check_clusters(ctx, shape, n_clusters));
+  if (n_iters < 1 || n_iters > 1000) return fail(ctx, ISA_ERR_INVALID_ARG, "n_iters = %d: need 1..1000", n_iters);
+  ISA_TRY(check_ptr(ctx, x, "x", 16));
+  ISA_TRY(check_ptr(ctx, centroids, "centroids", 16));
+  ISA_TRY(check_ptr(ctx, labels, "labels", 4));
+  ISA_TRY(check_ptr(ctx, perm, "perm", 4));
+  ISA_TRY(check_ptr(ctx, offsets, "offsets", 4));
+  if ((groups == nullptr) != (n_groups == nullptr))
+    return fail(ctx, ISA_ERR_INVALID_ARG, "groups and n_groups are given together or not at all");
+  if (groups) {
+    ISA_TRY(check_ptr(ctx, groups, "groups", 4));
+    ISA_TRY(check_ptr(ctx, n_groups, "n_groups", 4));
+  }
+  ISA_TRY(check_ptr(ctx, workspace, "workspace", 16));
+  if (workspace_bytes < cluster_ws(shape, n_clusters))
+    return fail(ctx, ISA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes,
+                cluster_ws(shape, n_clusters));
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ClusterLaunch l = cluster_launch(shape, n_clusters, x, centroids, workspace);
+  l.labels = labels;
+  l.perm = perm;
+  l.offsets = offsets;
+  ISA_TRY(cuda_status(ctx, launch_cluster_init(l, st), "isa_cluster"));
+  for (int it = 0; it < n_iters; ++it) {
+    const bool last = it == n_iters - 1;
+    l.groups = last ? groups : nullptr;
+    l.n_groups = last ? n_groups : nullptr;
+    ISA_TRY(cuda_status(ctx, launch_cluster_assign(l, st), "isa_cluster"));
+    ISA_TRY(cuda_status(ctx, launch_cluster_sort(l, ctx->d_status, st), "isa_cluster"));
+    ISA_TRY(cuda_status(ctx, launch_cluster_update(l, st), "isa_cluster"));
+  }
+  return ISA_OK;
+}
+
+isa_status isa_cluster_assign(isa_context* ctx, const isa_shape* shape, const void* x, const float* centroids,
+                              int32_t n_clusters, int32_t* labels, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  ISA_TRY(check_rows_shape(ctx, shape));
+  ISA_TRY(check_clusters(ctx, shape, n_clusters));
+  ISA_TRY(check_ptr(ctx, x, "x", 16));
+  ISA_TRY(check_ptr(ctx, centroids, "centroids", 4));
+  ISA_TRY(check_ptr(ctx, labels, "labels", 4));
+  ISA_TRY(check_ptr(ctx, workspace, "workspace", 16));
+  if (workspace_bytes < cluster_ws(shape, n_clusters))
+    return fail(ctx, ISA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes,
+                cluster_ws(shape, n_clusters));
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ClusterLaunch l = cluster_launch(shape, n_clusters, x, const_cast<float*>(centroids), workspace);
+  l.labels = labels;
+  ISA_TRY(cuda_status(ctx, launch_cluster_prep(l, st), "isa_cluster_assign"));
+  return cuda_status(ctx, launch_cluster_assign(l, st), "isa_cluster_assign");
+}
+
+isa_status isa_cluster_sort(isa_context* ctx, const isa_shape* shape, const int32_t* labels, int32_t n_clusters,
+                            int32_t* perm, int32_t* offsets, int32_t* groups, int32_t* n_groups, void* stream) {
+  ISA_TRY(check_rows_shape(ctx, shape));
+  ISA_TRY(check_clusters(ctx, shape, n_clusters));
+  ISA_TRY(check_ptr(ctx, labels, "labels", 4));
+  ISA_TRY(check_ptr(ctx, perm, "perm", 4));
+  ISA_TRY(check_ptr(ctx, offsets, "offsets", 4));
+  if ((groups == nullptr) != (n_groups == nullptr))
+    return fail(ctx, ISA_ERR_INVALID_ARG, "groups and n_groups are given together or not at all");
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  ClusterLaunch l{};
+  l.BH = shape->batch * shape->heads;
+  l.N = shape->seq_len;
+  l.D = shape->head_dim;
+  l.C = n_clusters;
+  l.labels = const_cast<int32_t*>(labels);
+  l.perm = perm;
+  l.offsets = offsets;
+  l.groups = groups;
+  l.n_groups = n_groups;
+  return cuda_status(ctx, launch_cluster_sort(l, ctx->d_status, static_cast<cudaStream_t>(stream)),
+                     "isa_cluster_sort");
+}
+
+isa_status isa_cluster_update(isa_context* ctx, const isa_shape* shape, const void* x, const int32_t* perm,
+                              const int32_t* offsets, int32_t n_clusters, float* centroids, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  ISA_TRY(check_rows_shape(ctx, shape));
+  ISA_TRY(check_clusters(ctx, shape, n_clusters));
+  ISA_TRY(check_ptr(ctx, x, "x", 16));
+  ISA_TRY(check_ptr(ctx, perm, "perm", 4));
+  ISA_TRY(check_ptr(ctx, offsets, "offsets", 4));
+  ISA_TRY(check_ptr(ctx, centroids, "centroids", 16));
+  ISA_TRY(check_ptr(ctx, workspace, "workspace", 16));
+  if (workspace_bytes < cluster_ws(shape, n_clusters))
+    return fail(ctx, ISA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes,
+                cluster_ws(shape, n_clusters));
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  ClusterLaunch l = cluster_launch(shape, n_clusters, x, centroids, workspace);
+  l.perm = const_cast<int32_t*>(perm);
+  l.offsets = const_cast<int32_t*>(offsets);
+  return cuda_status(ctx, launch_cluster_update(l, static_cast<cudaStream_t>(stream)), "isa_cluster_update");
+}
+
+isa_status isa_permute_rows(isa_context* ctx, const isa_shape* shape, const void* x, const int32_t* perm,
+                            int32_t inverse, void* out, void* stream) {
+  ISA_TRY(check_rows_shape(ctx, shape));
+  ISA_TRY(check_ptr(ctx, x, "x", 16));
+  ISA_TRY(check_ptr(ctx, perm, "perm", 4));
+  ISA_TRY(check_ptr(ctx, out, "out", 16));
+  if (x == out) return fail(ctx, ISA_ERR_INVALID_ARG, "x and out must not be the same buffer");
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  return cuda_status(ctx,
+                     launch_permute_rows(x, perm, shape->batch * shape->heads, shape->seq_len, shape->head_dim,
+                                         inverse != 0, out, ctx->d_status, ctx->num_sms,
+                                         static_cast<cudaStream_t>(stream)),
+                     "isa_permute_rows");
 }
 
 size_t isa_attention_workspace_bytes(const isa_shape* s) { return s ? attn_ws_bytes(s) : 0; }

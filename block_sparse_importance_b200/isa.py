@@ -68,6 +68,13 @@ def lib():
             L.isa_score.argtypes = [_P, S, _P, _P, _i32, _i32, _P, _P, _P, _P, _sz, _P]
             L.isa_select.argtypes = [_P, S, _P, _i32, _i32, _u64, _P, _P, _P]
             L.isa_select_top_p.argtypes = [_P, S, _P, ctypes.c_double, _i32, _u64, _P, _P, _P, _P]
+            L.isa_cluster_workspace_bytes.argtypes = [S, _i32]
+            L.isa_cluster_workspace_bytes.restype = _sz
+            L.isa_cluster.argtypes = [_P, S, _P, _i32, _i32, _P, _P, _P, _P, _P, _P, _P, _sz, _P]
+            L.isa_cluster_assign.argtypes = [_P, S, _P, _P, _i32, _P, _P, _sz, _P]
+            L.isa_cluster_sort.argtypes = [_P, S, _P, _i32, _P, _P, _P, _P, _P]
+            L.isa_cluster_update.argtypes = [_P, S, _P, _P, _P, _i32, _P, _P, _sz, _P]
+            L.isa_permute_rows.argtypes = [_P, S, _P, _P, _i32, _P, _P]
             L.isa_attention_workspace_bytes.argtypes = [S]
             L.isa_attention_workspace_bytes.restype = _sz
             L.isa_attention.argtypes = [_P, S, _P, _P, _P, _P, _P, _i32, _P, _P, _P, _sz, _P]
@@ -82,7 +89,9 @@ def lib():
             L.isa_debug_set.restype = ctypes.c_int
             L.isa_attention_noalloc.argtypes = [_P, S, _P, _P, _P, _P, _P, _i32, _P, _P, _P]
             for name in ("isa_create", "isa_sync_status", "isa_score", "isa_select", "isa_select_top_p", "isa_attention",
-                         "isa_dense_attention", "isa_pipeline", "isa_pipeline_host", "isa_attention_noalloc"):
+                         "isa_dense_attention", "isa_pipeline", "isa_pipeline_host", "isa_attention_noalloc",
+                         "isa_cluster", "isa_cluster_assign", "isa_cluster_sort", "isa_cluster_update",
+                         "isa_permute_rows"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -256,6 +265,102 @@ def select_top_p(mass, lay: Layout, top_p: float, n_select: int, seed: int, idx=
                                 ctypes.c_uint64(seed), _ptr(idx), _ptr(log_w), _ptr(n_exact), _stream(stream))
     ctx.check(st, "isa_select_top_p")
     return idx, log_w, n_exact
+
+
+def _rows_shape(x: torch.Tensor) -> Shape:
+    """isa_shape of the token-clustering calls (batch, heads, seq_len, head_dim)."""
+    B, H, N, d = x.shape
+    return Shape(B, H, N, d, 1, 64, N, None, 1.0)
+
+
+def cluster_workspace_bytes(x: torch.Tensor, n_clusters: int) -> int:
+    return int(lib().isa_cluster_workspace_bytes(ctypes.byref(_rows_shape(x)), n_clusters))
+
+
+def cluster(x, n_clusters: int, n_iters: int, workspace=None, ctx: Optional[Context] = None, stream=None):
+    """isa_cluster: k-means of every (batch, head) over the whole sequence and
+    the stable sort of its labels.  Returns a dict of device tensors:
+    centroids [B,H,C,d] f32, labels / perm [B,H,N] i32, offsets / groups
+    [B,H,C+1] i32 and n_groups [B,H] i32."""
+    ctx = ctx or context(x.device.index or 0)
+    _dev(x, torch.bfloat16, "x")
+    B, H, N, d = x.shape
+    C = n_clusters
+    r = {"centroids": _empty((B, H, C, d), torch.float32, x.device),
+         "labels": _empty((B, H, N), torch.int32, x.device),
+         "perm": _empty((B, H, N), torch.int32, x.device),
+         "offsets": _empty((B, H, C + 1), torch.int32, x.device),
+         "groups": _empty((B, H, C + 1), torch.int32, x.device),
+         "n_groups": _empty((B, H), torch.int32, x.device)}
+    sh = _rows_shape(x)
+    nb = int(lib().isa_cluster_workspace_bytes(ctypes.byref(sh), C))
+    ws = _workspace(nb, x.device, workspace)
+    st = lib().isa_cluster(ctx.handle, ctypes.byref(sh), _ptr(x), C, n_iters, _ptr(r["centroids"]), _ptr(r["labels"]),
+                           _ptr(r["perm"]), _ptr(r["offsets"]), _ptr(r["groups"]), _ptr(r["n_groups"]), _ptr(ws), nb,
+                           _stream(stream))
+    ctx.check(st, "isa_cluster")
+    return r
+
+
+def cluster_assign(x, centroids, workspace=None, ctx: Optional[Context] = None, stream=None):
+    """isa_cluster_assign: nearest of the given centroids [B,H,C,d] f32 -> labels [B,H,N] i32."""
+    ctx = ctx or context(x.device.index or 0)
+    _dev(x, torch.bfloat16, "x")
+    _dev(centroids, torch.float32, "centroids")
+    C = centroids.shape[2]
+    labels = _empty(x.shape[:3], torch.int32, x.device)
+    sh = _rows_shape(x)
+    nb = int(lib().isa_cluster_workspace_bytes(ctypes.byref(sh), C))
+    ws = _workspace(nb, x.device, workspace)
+    st = lib().isa_cluster_assign(ctx.handle, ctypes.byref(sh), _ptr(x), _ptr(centroids), C, _ptr(labels), _ptr(ws),
+                                  nb, _stream(stream))
+    ctx.check(st, "isa_cluster_assign")
+    return labels
+
+
+def cluster_sort(labels, n_clusters: int, head_dim: int = 128, ctx: Optional[Context] = None, stream=None):
+    """isa_cluster_sort: labels [B,H,N] i32 -> (perm, offsets, groups, n_groups)."""
+    ctx = ctx or context(labels.device.index or 0)
+    _dev(labels, torch.int32, "labels")
+    B, H, N = labels.shape
+    C = n_clusters
+    perm = _empty((B, H, N), torch.int32, labels.device)
+    off = _empty((B, H, C + 1), torch.int32, labels.device)
+    grp = _empty((B, H, C + 1), torch.int32, labels.device)
+    ng = _empty((B, H), torch.int32, labels.device)
+    sh = Shape(B, H, N, head_dim, 1, 64, N, None, 1.0)
+    st = lib().isa_cluster_sort(ctx.handle, ctypes.byref(sh), _ptr(labels), C, _ptr(perm), _ptr(off), _ptr(grp),
+                                _ptr(ng), _stream(stream))
+    ctx.check(st, "isa_cluster_sort")
+    return perm, off, grp, ng
+
+
+def cluster_update(x, perm, offsets, centroids, workspace=None, ctx: Optional[Context] = None, stream=None):
+    """isa_cluster_update: centroids [B,H,C,d] f32 updated in place to the
+    means of the sorted clusters (empty clusters keep theirs)."""
+    ctx = ctx or context(x.device.index or 0)
+    _dev(x, torch.bfloat16, "x")
+    _dev(centroids, torch.float32, "centroids")
+    C = centroids.shape[2]
+    sh = _rows_shape(x)
+    nb = int(lib().isa_cluster_workspace_bytes(ctypes.byref(sh), C))
+    ws = _workspace(nb, x.device, workspace)
+    st = lib().isa_cluster_update(ctx.handle, ctypes.byref(sh), _ptr(x), _ptr(perm), _ptr(offsets), C,
+                                  _ptr(centroids), _ptr(ws), nb, _stream(stream))
+    ctx.check(st, "isa_cluster_update")
+    return centroids
+
+
+def permute_rows(x, perm, inverse: bool = False, out=None, ctx: Optional[Context] = None, stream=None):
+    """isa_permute_rows: out[i] = x[perm[i]], or out[perm[i]] = x[i] with inverse."""
+    ctx = ctx or context(x.device.index or 0)
+    _dev(x, torch.bfloat16, "x")
+    _dev(perm, torch.int32, "perm")
+    out = out if out is not None else _empty(x.shape, torch.bfloat16, x.device)
+    st = lib().isa_permute_rows(ctx.handle, ctypes.byref(_rows_shape(x)), _ptr(x), _ptr(perm), 1 if inverse else 0,
+                                _ptr(out), _stream(stream))
+    ctx.check(st, "isa_permute_rows")
+    return out
 
 
 def attention(q, k, v, idx, log_w, lay: Layout, out=None, lse=None, workspace=None,

@@ -187,6 +187,71 @@ ISA_API isa_status isa_select_top_p(isa_context* ctx, const isa_shape* shape, co
                             float* log_w, int32_t* n_exact_rows, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Token clustering: the permuted layout of permuted block-sparse attention
+ * ("InstaGen", abstract: PBSA computes blocks of a semantically permuted
+ * attention matrix, and InstaGen is parameterised by SVG2, whose
+ * semantic-aware permutation clusters the tokens of the whole sequence;
+ * "AB-Attention" names that sequence-wide clustering and permutation as the
+ * cost its in-block clustering avoids).  Per (batch, head), Lloyd's k-means
+ * over all N rows of x with C clusters:
+ *   init    mu_c = row floor(c N / C);
+ *   assign  label_r = argmin_c ||x_r - mu_c||^2, ties to the lower c;
+ *   sort    perm = the rows in (label, row) order (a stable counting sort);
+ *           offsets[c] .. offsets[c+1] are cluster c's positions in perm;
+ *   update  mu_c = mean of cluster c's rows (an empty cluster keeps mu_c);
+ * n_iters rounds of (assign, sort, update); the labels, perm and offsets of
+ * the last round are returned with the centroids after its update.  A query
+ * cluster is one query group of the attention calls (q permuted by perm,
+ * q_offsets = that head's groups, out un-permuted by isa_permute_rows with
+ * inverse = 1); keys permuted by their own clustering form the key blocks.
+ * Only batch, heads, seq_len and head_dim of `shape` are read; x is
+ * [B,H,N,d] bf16.  The distances use x exact in bf16 and mu split into bf16
+ * hi + lo parts (relative error 2^-16), so an assignment decided by a margin
+ * below ~3e-5 of ||x||^2 + ||mu||^2 may differ from an exact computation.
+ * ------------------------------------------------------------------------- */
+/* Scratch for isa_cluster / isa_cluster_assign / isa_cluster_update: the
+ * centroids' bf16 hi / lo parts and squared norms (C rounded up to 64).
+ * 0 for an invalid shape. */
+ISA_API size_t isa_cluster_workspace_bytes(const isa_shape* shape, int32_t n_clusters);
+
+/* The whole clustering.  1 <= n_clusters <= min(N, 8192), 1 <= n_iters <=
+ * 1000.  centroids: [B,H,C,d] fp32 (written).  labels, perm: [B,H,N] int32
+ * (written).  offsets: [B,H,C+1] int32 (written).  groups: optional
+ * [B,H,C+1] int32, the offsets of the non-empty clusters only, and
+ * n_groups: [B,H] int32 their count (both NULL, or both given).  workspace:
+ * isa_cluster_workspace_bytes bytes, 16-byte aligned. */
+ISA_API isa_status isa_cluster(isa_context* ctx, const isa_shape* shape, const void* x, int32_t n_clusters,
+                       int32_t n_iters, float* centroids, int32_t* labels, int32_t* perm,
+                       int32_t* offsets, int32_t* groups, int32_t* n_groups, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* One assignment round against given centroids ([B,H,C,d] fp32, read). */
+ISA_API isa_status isa_cluster_assign(isa_context* ctx, const isa_shape* shape, const void* x,
+                              const float* centroids, int32_t n_clusters, int32_t* labels,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* The stable counting sort of given labels ([B,H,N] int32 in [0, C); a
+ * label outside it is skipped and sets ISA_ERR_DEVICE_CHECK). */
+ISA_API isa_status isa_cluster_sort(isa_context* ctx, const isa_shape* shape, const int32_t* labels,
+                            int32_t n_clusters, int32_t* perm, int32_t* offsets, int32_t* groups,
+                            int32_t* n_groups, void* stream);
+
+/* The mean update from a sorted layout (perm, offsets as isa_cluster_sort
+ * writes them); centroids are read (the empty clusters' rows) and written. */
+ISA_API isa_status isa_cluster_update(isa_context* ctx, const isa_shape* shape, const void* x,
+                              const int32_t* perm, const int32_t* offsets, int32_t n_clusters,
+                              float* centroids, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* Rows of d bf16 values, per (batch, head): out[i] = x[perm[i]] (inverse =
+ * 0, gather) or out[perm[i]] = x[i] (inverse = 1, scatter).  x, out:
+ * [B,H,N,d], distinct buffers, 16-byte aligned; perm: [B,H,N], a
+ * permutation of 0..N-1 (an index outside it is skipped and sets
+ * ISA_ERR_DEVICE_CHECK). */
+ISA_API isa_status isa_permute_rows(isa_context* ctx, const isa_shape* shape, const void* x,
+                            const int32_t* perm, int32_t inverse, void* out, void* stream);
+
+/* ---------------------------------------------------------------------------
  * isa_attention -- one sparse flash-attention pass over a plan
  * ("AB-Attention": the weights become shifts of the sampled blocks' scores
  * before the softmax, and only selected blocks receive exact attention; small

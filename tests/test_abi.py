@@ -18,7 +18,9 @@ def test_header_declares_the_boundary():
     names = isa.declared_symbols()
     for n in ["isa_create", "isa_destroy", "isa_score", "isa_select", "isa_select_top_p", "isa_attention",
               "isa_dense_attention", "isa_sync_status", "isa_status_string", "isa_score_workspace_bytes",
-              "isa_attention_workspace_bytes", "isa_pipeline", "isa_pipeline_host"]:
+              "isa_attention_workspace_bytes", "isa_pipeline", "isa_pipeline_host", "isa_cluster",
+              "isa_cluster_assign", "isa_cluster_sort", "isa_cluster_update", "isa_cluster_workspace_bytes",
+              "isa_permute_rows"]:
         assert n in names
 
 
@@ -65,3 +67,12 @@ def test_create_fails_cleanly_without_a_gpu(L):
     h = ctypes.c_void_p()
     assert L.isa_create(0, ctypes.byref(h)) != isa.ISA_OK
     assert not h.value
+
+
+def test_cluster_workspace_size(L):
+    import torch
+    x = torch.empty(1, 40, 75600, 128, dtype=torch.bfloat16, device="meta")
+    up = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    cp = 640  # 600 clusters rounded up to 64
+    assert isa.cluster_workspace_bytes(x, 600) == 2 * up(40 * cp * 128 * 2) + up(40 * cp * 4)
+    assert isa.cluster_workspace_bytes(x, 0) == 0
