@@ -249,6 +249,8 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--top-p", type=float, default=0.0,
+                    help="also time isa_select_top_p (exact set by a share of the mass) on the step's mass")
     ap.add_argument("--cluster", type=int, default=0,
                     help="also time the permuted layout's build: isa_cluster of Q and of K with this many clusters "
                          "(3 rounds) and the row permutations of Q, K and V")
@@ -372,6 +374,30 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         dense_ms = e0.elapsed_time(e1) / 2
+
+    # the top-p selector on the same mass (count kernel + selector): mass read
+    # twice, plan and per-row exact-set sizes written
+    if rank == 0 and args.top_p > 0.0:
+        ne_rows = torch.empty(B, H, G, dtype=torch.int32, device=dev)
+        isa.select_top_p(mass, lay, args.top_p, S, w.seed, idx=idx, log_w=lw, n_exact=ne_rows, ctx=ctx)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            isa.select_top_p(mass, lay, args.top_p, S, w.seed, idx=idx, log_w=lw, n_exact=ne_rows, ctx=ctx)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        st = ctx.sync_status()
+        if st != isa.ISA_OK:
+            raise RuntimeError("device status after the top-p selector: %s" % isa.status_string(st))
+        tp_ms = e0.elapsed_time(e1) / 3
+        tp_bytes = B * H * G * (8 * nK + 8 * S + 4)
+        ke = ne_rows.float()
+        stages["select_top_p"] = {"ms": tp_ms, "p": args.top_p, "bytes": tp_bytes,
+                                  "gbs": tp_bytes / (tp_ms * 1e-3) / 1e9,
+                                  "frac_hbm": tp_bytes / (tp_ms * 1e-3) / 1e9 / hbm,
+                                  "n_exact_mean": float(ke.mean()), "n_exact_min": int(ke.min()),
+                                  "n_exact_max": int(ke.max())}
+        del ne_rows
 
     # the permuted layout's build (token clustering of Q and K, then the row
     # permutations): algorithmic FLOPs are the distance products, 2 N C d per

@@ -9,9 +9,9 @@
 // and token permutation.  Per (batch, head), Lloyd's k-means over all N rows
 // with C clusters, centroids initialised at rows floor(c N / C); each round
 //   assign  argmin_c ||x - mu_c||^2 = argmin_c (|mu_c|^2 - 2 x.mu_c), ties to
-//           the lower c; the dot products run on tensor cores (mma.sync
-//           m16n8k16) with x exact in bf16 and mu split into bf16 hi + lo
-//           parts (relative error 2^-16), two products per tile;
+//           the lower c; the dot products run on the tensor cores (tcgen05,
+//           fp32 accumulators in TMEM) with x exact in bf16 and mu split into
+//           bf16 hi + lo parts (relative error 2^-16), two products per k-step;
 //   sort    a stable counting sort of the labels: perm lists the rows in
 //           (label, row) order, offsets[c] .. offsets[c + 1] are cluster c's;
 //   update  mu_c = the fp32 mean of cluster c's rows taken in permutation
@@ -27,27 +27,14 @@
 #include "isa_internal.h"
 #include "mma_sync.cuh"
 #include "ptx.cuh"
+#include "tmap.h"
 
 namespace isa_impl {
 namespace {
 
 __device__ __forceinline__ float bf16f(uint16_t h) { return __uint_as_float(static_cast<uint32_t>(h) << 16); }
 
-constexpr int kAsgThreads = 128;  // 4 warps x 32 rows
-constexpr int kAsgRows = 128;
-constexpr int kAsgChunk = 64;     // centroids per shared-memory stage
 constexpr int kPrepWarps = 8;
-
-template <int D>
-struct AsgLayout {
-  static constexpr int XS = D + 8;  // padded row (elements): ldmatrix rows land in distinct banks
-  static constexpr uint32_t kX = 0;
-  static constexpr uint32_t kXBytes = kAsgRows * XS * 2;
-  static constexpr uint32_t kStageBytes = 2 * kAsgChunk * XS * 2;  // hi rows, then lo rows
-  static constexpr uint32_t kC = kXBytes;
-  static constexpr uint32_t kN = kC + 2 * kStageBytes;
-  static constexpr uint32_t kAlloc = kN + 2 * kAsgChunk * 4;
-};
 
 // mu_c = row floor(c N / C) of the head, as fp32.  One warp per centroid.
 template <int D>
@@ -101,141 +88,236 @@ __global__ void __launch_bounds__(kPrepWarps * 32) cluster_prep_kernel(ClusterLa
   write_prep<D>(l, bh, c, v, live);
 }
 
-// Nearest centroid of 128 rows per CTA.  The rows sit in shared memory and,
-// as mma A fragments, in registers (two 16-row tiles per warp); centroids
-// stream through a two-stage cp.async ring 64 at a time.  Within a lane the
-// candidates come in ascending c and a strict compare keeps the first
-// minimum; across the quad, equal distances go to the lower c.
+// Nearest centroid on the tensor cores (tcgen05), a persistent CTA per SM
+// walking 128-row tiles of the heads.  Per tile, the centroids come in chunks
+// of 128; for each chunk the MMA warp computes S = X hi^T + X lo^T (M = 128
+// rows, N = 128 centroids, K = d; two products per k-step) into one of two
+// TMEM accumulators, and each epilogue thread (one per row = TMEM lane)
+// updates its running argmin of nsq_c - 2 S_c.  Candidates arrive in
+// ascending c and a strict compare keeps the first minimum, so ties go to
+// the lower c with no cross-lane step.
+//   warps 0-3  epilogue (argmin, labels);
+//   warp 4     TMA producer: the X tile (two buffers) and the centroid hi / lo
+//              chunks (two stages);
+//   warp 5     MMA issue (one elected lane of a converged warp).
+// Every wait is bounded (global timer + CTA abort flag): on a timeout the CTA
+// drains its copies and products, frees TMEM and records ISA_ERR_TIMEOUT.
+constexpr int kAsgThreads = 192;
+constexpr int kAsgRows = 128;
+constexpr int kAsgChunk = 128;  // centroids per stage (the MMA's N)
+
 template <int D>
-__global__ void __launch_bounds__(kAsgThreads) cluster_assign_kernel(ClusterLaunch l) {
+struct AsgLayout {
+  static constexpr uint32_t kTile = 128 * D * 2;  // 128 rows x D bf16, 64-column boxes, 128-byte swizzle
+  static constexpr uint32_t kBox = 128 * 128;     // one 64-column box of 128 rows
+  static constexpr uint32_t kX = 0;               // two X buffers
+  static constexpr uint32_t kRing = 2 * kTile;    // two stages of (hi, lo)
+  static constexpr uint32_t kStage = 2 * kTile;
+  static constexpr uint32_t kNsq = kRing + 2 * kStage;  // 4 warps x 128 floats
+  static constexpr uint32_t kBar = kNsq + 4 * kAsgChunk * 4;
+  static constexpr int kXFull = 0, kXEmpty = 2, kFull = 4, kEmpty = 6, kAFull = 8, kAEmpty = 10, kFinal = 12,
+                       kNumBars = 13;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8;
+  static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAsgThreads, 1)
+    cluster_assign_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_hi,
+                          const __grid_constant__ CUtensorMap tm_lo, ClusterLaunch l, uint64_t timeout_ns,
+                          int* status) {
   using namespace isa_dev;
   using L = AsgLayout<D>;
-  constexpr int XS = L::XS, KSTEPS = D / 16;
-  extern __shared__ __align__(16) uint8_t sm[];
-  const uint32_t sbase = smem_addr(sm);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-  const int64_t bh = blockIdx.y;
-  const int r0 = blockIdx.x * kAsgRows;
-  const int rows = min(kAsgRows, l.N - r0);
-  const uint16_t* xg = static_cast<const uint16_t*>(l.x) + (bh * l.N + r0) * D;
-  for (int i = tid; i < kAsgRows * (D / 8); i += kAsgThreads) {
-    const int r = i / (D / 8), c16 = i - r * (D / 8);
-    const bool in = r < rows;
-    cp_async16_zfill(sbase + L::kX + 2u * (r * XS + c16 * 8), in ? xg + static_cast<int64_t>(r) * D + c16 * 8 : xg,
-                     in ? 16u : 0u);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + L::kBar + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tiles_per_head = (l.N + kAsgRows - 1) / kAsgRows;
+  const int64_t n_tiles = static_cast<int64_t>(l.BH) * tiles_per_head;
+  const int nch = l.Cpad / kAsgChunk;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::kXFull + i), 1);
+      mbar_init(bar(L::kXEmpty + i), 1);
+      mbar_init(bar(L::kFull + i), 1);
+      mbar_init(bar(L::kEmpty + i), 1);
+      mbar_init(bar(L::kAFull + i), 1);
+      mbar_init(bar(L::kAEmpty + i), 128);
+    }
+    mbar_init(bar(L::kFinal), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  const uint16_t* hig = l.mu_hi + bh * l.Cpad * D;
-  const uint16_t* lowg = l.mu_lo + bh * l.Cpad * D;
-  const float* nsg = l.mu_nsq + bh * l.Cpad;
-  auto load_stage = [&](int ch, int st) {
-    const uint32_t dst = sbase + L::kC + st * L::kStageBytes;
-    for (int i = tid; i < kAsgChunk * (D / 8); i += kAsgThreads) {
-      const int r = i / (D / 8), c16 = i - r * (D / 8);
-      const int64_t src = static_cast<int64_t>(ch * kAsgChunk + r) * D + c16 * 8;
-      cp_async16(dst + 2u * (r * XS + c16 * 8), hig + src);
-      cp_async16(dst + 2u * ((kAsgChunk + r) * XS + c16 * 8), lowg + src);
-    }
-    if (tid < kAsgChunk / 4) cp_async16(sbase + L::kN + st * kAsgChunk * 4 + tid * 16, nsg + ch * kAsgChunk + tid * 4);
-  };
-  const int n_chunks = l.Cpad / kAsgChunk;
-  load_stage(0, 0);
-  cp_async_commit();
-  // ldmatrix lane addresses: A tile (rows, k) and a pair of B n-tiles
-  // (matrices: n 0-7 k 0-7, n 0-7 k 8-15, n 8-15 k 0-7, n 8-15 k 8-15)
-  const int a_row = (lane & 7) + ((lane >> 3) & 1) * 8, a_col = (lane >> 4) * 8;
-  const int b_row = (lane & 7) + (lane >> 4) * 8, b_col = ((lane >> 3) & 1) * 8;
-  uint32_t a[2][KSTEPS][4];
-  float best[2][2];
-  int bi[2][2];
+  if (warp == 5) {
+    tmem_alloc(smem_addr(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t item = 0, tc = 0, issued = 0, x_issued = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tc) {
+        const int bh = static_cast<int>(t / tiles_per_head);
+        const int row = static_cast<int>(t - static_cast<int64_t>(bh) * tiles_per_head) * kAsgRows;
+        const uint32_t xb = tc & 1u;
+        if (!mbar_wait(bar(L::kXEmpty + xb), ((tc >> 1) & 1u) ^ 1u, abort_flag, timeout_ns)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(L::kXFull + xb), L::kTile);
 #pragma unroll
-  for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(base + L::kX + xb * L::kTile + c * L::kBox, &tm_x, bar(L::kXFull + xb), c * 64, row, bh);
+        ++x_issued;
+        for (int j = 0; j < nch; ++j, ++item) {
+          const uint32_t s = item & 1u;
+          if (!mbar_wait(bar(L::kEmpty + s), ((item >> 1) & 1u) ^ 1u, abort_flag, timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(L::kFull + s), L::kStage);
+          const uint32_t dst = base + L::kRing + s * L::kStage;
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      best[t][hh] = INFINITY;
-      bi[t][hh] = 0;
-    }
-  for (int ch = 0; ch < n_chunks; ++ch) {
-    const int st = ch & 1;
-    if (ch + 1 < n_chunks) {
-      load_stage(ch + 1, st ^ 1);
-      cp_async_commit();
-      cp_async_wait_group<1>();
-    } else {
-      cp_async_wait_group<0>();
-    }
-    __syncthreads();
-    if (ch == 0) {
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int ks = 0; ks < KSTEPS; ++ks)
-          ldsm_x4(a[t][ks], sbase + L::kX + 2u * ((32 * warp + 16 * t + a_row) * XS + ks * 16 + a_col));
-    }
-    const uint32_t hi_s = sbase + L::kC + st * L::kStageBytes, lo_s = hi_s + kAsgChunk * XS * 2;
-    const float* ns = reinterpret_cast<const float*>(sm + L::kN) + st * kAsgChunk;
-#pragma unroll 1
-    for (int np = 0; np < kAsgChunk / 16; ++np) {
-      float acc[2][2][4];
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc[t][j][k] = 0.0f;
-#pragma unroll
-      for (int ks = 0; ks < KSTEPS; ++ks) {
-        uint32_t bh4[4], bl4[4];
-        const uint32_t off = 2u * ((np * 16 + b_row) * XS + ks * 16 + b_col);
-        ldsm_x4(bh4, hi_s + off);
-        ldsm_x4(bl4, lo_s + off);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) mma_16816(acc[t][j], a[t][ks], bh4[2 * j], bh4[2 * j + 1]);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) mma_16816(acc[t][j], a[t][ks], bl4[2 * j], bl4[2 * j + 1]);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_3d(dst + c * L::kBox, &tm_hi, bar(L::kFull + s), c * 64, j * kAsgChunk, bh);
+            tma_load_3d(dst + L::kTile + c * L::kBox, &tm_lo, bar(L::kFull + s), c * 64, j * kAsgChunk, bh);
+          }
+          ++issued;
+        }
       }
+      if (!ok || *abort_flag) {
+        // let the copies already issued land before the CTA leaves
+        const uint32_t first = issued > 2 ? issued - 2 : 0;
+        for (uint32_t i = first; i < issued; ++i) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(bar(L::kFull + (i & 1u)), (i >> 1) & 1u))
+            if (global_timer_ns() - t0 > 200000000ull) break;
+        }
+        const uint32_t xfirst = x_issued > 2 ? x_issued - 2 : 0;
+        for (uint32_t i = xfirst; i < x_issued; ++i) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(bar(L::kXFull + (i & 1u)), (i >> 1) & 1u))
+            if (global_timer_ns() - t0 > 200000000ull) break;
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ----------------------------------------------------------------- MMA
+    constexpr uint32_t idesc = idesc_bf16_f32(128, kAsgChunk, 0);
+    const uint64_t dx = smem_desc_sw128(base + L::kX, 16, 1024);
+    const uint64_t dr = smem_desc_sw128(base + L::kRing, 16, 1024);
+    uint32_t item = 0, tc = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tc) {
+      const uint32_t xb = tc & 1u;
+      if (!mbar_wait_warp(bar(L::kXFull + xb), (tc >> 1) & 1u, abort_flag, timeout_ns)) break;
+      const uint64_t a0 = dx + ((xb * L::kTile) >> 4);
+      for (int j = 0; j < nch; ++j, ++item) {
+        const uint32_t s = item & 1u, ab = item & 1u;
+        if (!mbar_wait_warp(bar(L::kFull + s), (item >> 1) & 1u, abort_flag, timeout_ns) ||
+            !mbar_wait_warp(bar(L::kAEmpty + ab), ((item >> 1) & 1u) ^ 1u, abort_flag, timeout_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t b_hi = dr + ((s * L::kStage) >> 4), b_lo = b_hi + (L::kTile >> 4);
+        const uint32_t d = tmem + ab * kAsgChunk;
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t off = ((k >> 2) * L::kBox + (k & 3) * 32) >> 4;
+          if (elect_one()) mma_ss(d, a0 + off, b_hi + off, idesc, k > 0 ? 1u : 0u);
+          if (elect_one()) mma_ss(d, a0 + off, b_lo + off, idesc, 1u);
+        }
+        if (elect_one()) {
+          tc_commit(bar(L::kEmpty + s));
+          tc_commit(bar(L::kAFull + ab));
+          if (j == nch - 1) tc_commit(bar(L::kXEmpty + xb));
+        }
+      }
+    }
+    if (elect_one()) tc_commit(bar(L::kFinal));
+    __syncwarp();
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar(L::kFinal), 0))
+      if (global_timer_ns() - t0 > 200000000ull) break;
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int r = warp * 32 + lane;  // row of the tile == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float* nsq_s = reinterpret_cast<float*>(smem + L::kNsq) + warp * kAsgChunk;
+    // this lane's four norms of an item's chunk, fetched one item ahead
+    auto fetch = [&](int64_t t, int j) -> float4 {
+      const int bh = static_cast<int>(t / tiles_per_head);
+      return *reinterpret_cast<const float4*>(l.mu_nsq + static_cast<int64_t>(bh) * l.Cpad + j * kAsgChunk +
+                                              4 * lane);
+    };
+    uint32_t item = 0;
+    int64_t t = blockIdx.x;
+    float4 nq = t < n_tiles ? fetch(t, 0) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    bool ok = true;
+    for (; t < n_tiles && ok; t += gridDim.x) {
+      const int bh = static_cast<int>(t / tiles_per_head);
+      const int row0 = static_cast<int>(t - static_cast<int64_t>(bh) * tiles_per_head) * kAsgRows;
+      float best = INFINITY;
+      int bi = 0;
+      for (int j = 0; j < nch; ++j, ++item) {
+        __syncwarp();
+        *reinterpret_cast<float4*>(nsq_s + 4 * lane) = nq;
+        __syncwarp();
+        if (j + 1 < nch)
+          nq = fetch(t, j + 1);
+        else if (t + gridDim.x < n_tiles)
+          nq = fetch(t + gridDim.x, 0);
+        const uint32_t ab = item & 1u;
+        if (!mbar_wait(bar(L::kAFull + ab), (item >> 1) & 1u, abort_flag, timeout_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t v[4][32];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int cl = np * 16 + j * 8 + 2 * tq + e;
-          const float nsq = ns[cl];
-          const int c = ch * kAsgChunk + cl;
+        for (int cc = 0; cc < 4; ++cc) tmem_ld32(lane_base + ab * kAsgChunk + 32 * cc, v[cc]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(L::kAEmpty + ab));
 #pragma unroll
-          for (int t = 0; t < 2; ++t)
+        for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const float dist = nsq - 2.0f * acc[t][j][2 * hh + e];
-              if (dist < best[t][hh]) {
-                best[t][hh] = dist;
-                bi[t][hh] = c;
+          for (int e = 0; e < 32; e += 4) {
+            const float4 n4 = *reinterpret_cast<const float4*>(nsq_s + 32 * cc + e);
+            const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float dist = fmaf(-2.0f, __uint_as_float(v[cc][e + u]), nn[u]);
+              if (dist < best) {
+                best = dist;
+                bi = j * kAsgChunk + 32 * cc + e + u;
               }
             }
-        }
-    }
-    __syncthreads();  // every warp is done with this stage before it is refilled
-  }
-#pragma unroll
-  for (int t = 0; t < 2; ++t)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      float b = best[t][hh];
-      int i = bi[t][hh];
-#pragma unroll
-      for (int o = 1; o <= 2; o <<= 1) {
-        const float ob = __shfl_xor_sync(0xffffffffu, b, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, i, o);
-        if (ob < b || (ob == b && oi < i)) {
-          b = ob;
-          i = oi;
-        }
+          }
       }
-      const int r = 32 * warp + 16 * t + gq + 8 * hh;
-      if (tq == 0 && r < rows) l.labels[bh * l.N + r0 + r] = i;
+      if (ok && row0 + r < l.N) l.labels[static_cast<int64_t>(bh) * l.N + row0 + r] = bi;
     }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort_flag) atomicCAS(status, 0, kStatusTimeout);
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
 }
 
 // Stable counting sort of one head's labels, one warp per (batch, head):
@@ -243,9 +325,10 @@ __global__ void __launch_bounds__(kAsgThreads) cluster_assign_kernel(ClusterLaun
 // offsets of the non-empty clusters: the query groups), then the rows in
 // ascending order, 32 at a time: lanes with equal labels rank themselves by
 // lane order (__match_any_sync) and the lowest of them moves the cluster's
-// cursor.  Labels are read 32 x kSortBatch at a time, so that their loads
-// are in flight together.  A label outside [0, C) is skipped and sets the
-// device-check status (its row then has no place in perm).
+// cursor.  Labels are read 32 x kSortBatch at a time, a batch ahead of the
+// one being processed, so that their loads are in flight together.  A label
+// outside [0, C) is skipped and sets the device-check status (its row then
+// has no place in perm).
 constexpr int kSortBatch = 16;
 
 __global__ void __launch_bounds__(32) cluster_sort_kernel(ClusterLaunch l, int* status) {
@@ -256,14 +339,20 @@ __global__ void __launch_bounds__(32) cluster_sort_kernel(ClusterLaunch l, int* 
   const int32_t* lab = l.labels + bh * N;
   for (int c = lane; c < C; c += 32) cur[c] = 0;
   __syncwarp();
-  bool bad = false;
-  for (int base = 0; base < N; base += 32 * kSortBatch) {
-    int v[kSortBatch];
+  // labels of rows base + 32 k + lane, k < kSortBatch (-1 past N); the next
+  // batch's loads are issued before the current batch is processed
+  auto load_batch = [&](int base, int (&v)[kSortBatch]) {
 #pragma unroll
     for (int k = 0; k < kSortBatch; ++k) {
       const int r = base + 32 * k + lane;
       v[k] = r < N ? lab[r] : -1;
     }
+  };
+  bool bad = false;
+  int v[kSortBatch], nx[kSortBatch];
+  load_batch(0, v);
+  for (int base = 0; base < N; base += 32 * kSortBatch) {
+    if (base + 32 * kSortBatch < N) load_batch(base + 32 * kSortBatch, nx);
 #pragma unroll
     for (int k = 0; k < kSortBatch; ++k) {
       if (v[k] >= 0 && v[k] < C) {
@@ -272,6 +361,8 @@ __global__ void __launch_bounds__(32) cluster_sort_kernel(ClusterLaunch l, int* 
         bad = true;
       }
     }
+#pragma unroll
+    for (int k = 0; k < kSortBatch; ++k) v[k] = nx[k];
   }
   __syncwarp();
   // lane owns clusters [c0, c1)
@@ -309,17 +400,12 @@ __global__ void __launch_bounds__(32) cluster_sort_kernel(ClusterLaunch l, int* 
   }
   __syncwarp();
   int32_t* pm = l.perm + bh * N;
+  load_batch(0, v);
   for (int base = 0; base < N; base += 32 * kSortBatch) {
-    int v[kSortBatch];
+    if (base + 32 * kSortBatch < N) load_batch(base + 32 * kSortBatch, nx);
 #pragma unroll
     for (int k = 0; k < kSortBatch; ++k) {
-      const int r = base + 32 * k + lane;
-      const int c = r < N ? lab[r] : -1;
-      v[k] = (c >= 0 && c < C) ? c : -1;
-    }
-#pragma unroll
-    for (int k = 0; k < kSortBatch; ++k) {
-      const int c = v[k];
+      const int c = (v[k] >= 0 && v[k] < C) ? v[k] : -1;
       const unsigned peers = __match_any_sync(0xffffffffu, c);
       const int rank = __popc(peers & ((1u << lane) - 1u));
       const int pos = c >= 0 ? cur[c] + rank : 0;
@@ -330,6 +416,8 @@ __global__ void __launch_bounds__(32) cluster_sort_kernel(ClusterLaunch l, int* 
       }
       __syncwarp();
     }
+#pragma unroll
+    for (int k = 0; k < kSortBatch; ++k) v[k] = nx[k];
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(status, 0, kStatusDeviceCheck);
 }
@@ -433,8 +521,12 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __res
 }
 
 template <int D>
-int launch_assign_d(const ClusterLaunch& l, cudaStream_t stream) {
+int launch_assign_d(const ClusterLaunch& l, int num_sms, uint64_t timeout_ns, int* status, cudaStream_t stream) {
   using L = AsgLayout<D>;
+  CUtensorMap tx, thi, tlo;
+  if (!make_bf16_map(&tx, l.x, l.BH, l.N, D, 128) || !make_bf16_map(&thi, l.mu_hi, l.BH, l.Cpad, D, 128) ||
+      !make_bf16_map(&tlo, l.mu_lo, l.BH, l.Cpad, D, 128))
+    return -1;
   static bool attr = false;
   if (!attr) {
     const cudaError_t e = cudaFuncSetAttribute(cluster_assign_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -442,7 +534,9 @@ int launch_assign_d(const ClusterLaunch& l, cudaStream_t stream) {
     if (e != cudaSuccess) return static_cast<int>(e);
     attr = true;
   }
-  cluster_assign_kernel<D><<<dim3((l.N + kAsgRows - 1) / kAsgRows, l.BH), kAsgThreads, L::kAlloc, stream>>>(l);
+  const int64_t n_tiles = static_cast<int64_t>(l.BH) * ((l.N + kAsgRows - 1) / kAsgRows);
+  const int grid = static_cast<int>(n_tiles < num_sms ? n_tiles : num_sms);
+  cluster_assign_kernel<D><<<grid, kAsgThreads, L::kAlloc, stream>>>(tx, thi, tlo, l, timeout_ns, status);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -468,8 +562,11 @@ int launch_cluster_init(const ClusterLaunch& l, cudaStream_t stream) {
   return launch_cluster_prep(l, stream);
 }
 
-int launch_cluster_assign(const ClusterLaunch& l, cudaStream_t stream) {
-  return l.D == 128 ? launch_assign_d<128>(l, stream) : launch_assign_d<64>(l, stream);
+int launch_cluster_assign(const ClusterLaunch& l, int num_sms, uint64_t timeout_ns, int* status,
+                          cudaStream_t stream) {
+  const uint64_t t = timeout_ns ? timeout_ns : kWaitTimeoutNs;
+  return l.D == 128 ? launch_assign_d<128>(l, num_sms, t, status, stream)
+                    : launch_assign_d<64>(l, num_sms, t, status, stream);
 }
 
 int launch_cluster_sort(const ClusterLaunch& l, int* status, cudaStream_t stream) {

@@ -488,7 +488,7 @@ isa_status isa_cluster(isa_context* ctx, const isa_shape* shape, const void* x, 
     const bool last = it == n_iters - 1;
     l.groups = last ? groups : nullptr;
     l.n_groups = last ? n_groups : nullptr;
-    ISA_TRY(cuda_status(ctx, launch_cluster_assign(l, st), "isa_cluster"));
+    ISA_TRY(cuda_status(ctx, launch_cluster_assign(l, ctx->num_sms, ctx->wait_timeout_ns, ctx->d_status, st), "isa_cluster"));
     ISA_TRY(cuda_status(ctx, launch_cluster_sort(l, ctx->d_status, st), "isa_cluster"));
     ISA_TRY(cuda_status(ctx, launch_cluster_update(l, st), "isa_cluster"));
   }
@@ -513,7 +513,7 @@ isa_status isa_cluster_assign(isa_context* ctx, const isa_shape* shape, const vo
   ClusterLaunch l = cluster_launch(shape, n_clusters, x, const_cast<float*>(centroids), workspace);
   l.labels = labels;
   ISA_TRY(cuda_status(ctx, launch_cluster_prep(l, st), "isa_cluster_assign"));
-  return cuda_status(ctx, launch_cluster_assign(l, st), "isa_cluster_assign");
+  return cuda_status(ctx, launch_cluster_assign(l, ctx->num_sms, ctx->wait_timeout_ns, ctx->d_status, st), "isa_cluster_assign");
 }
 
 isa_status isa_cluster_sort(isa_context* ctx, const isa_shape* shape, const int32_t* labels, int32_t n_clusters,

@@ -84,7 +84,7 @@ int launch_score(const ScoreLaunch& s, cudaStream_t stream);
 // k-means over the whole sequence of every (batch, head) and the stable
 // counting sort of its labels (the permuted layout).  The centroids' bf16
 // hi / lo split and squared norms live in caller scratch, Cpad = C rounded
-// up to 64 rows (padding rows: zero, norm +inf).
+// up to 128 rows (padding rows: zero, norm +inf).
 struct ClusterLaunch {
   int BH, N, D, C, Cpad;
   const void* x;         // [BH, N, D] bf16
@@ -98,10 +98,11 @@ struct ClusterLaunch {
   int32_t* groups;       // [BH, C + 1] or NULL
   int32_t* n_groups;     // [BH] or NULL
 };
-inline int cluster_cpad(int C) { return (C + 63) / 64 * 64; }
+inline int cluster_cpad(int C) { return (C + 127) / 128 * 128; }
 int launch_cluster_init(const ClusterLaunch& l, cudaStream_t stream);     // mu = rows floor(c N / C), then prep
 int launch_cluster_prep(const ClusterLaunch& l, cudaStream_t stream);     // hi / lo / norms of mu
-int launch_cluster_assign(const ClusterLaunch& l, cudaStream_t stream);   // labels from hi / lo / norms
+int launch_cluster_assign(const ClusterLaunch& l, int num_sms, uint64_t timeout_ns, int* status,
+                          cudaStream_t stream);  // labels from hi / lo / norms (tcgen05)
 int launch_cluster_sort(const ClusterLaunch& l, int* status, cudaStream_t stream);  // perm, offsets (groups)
 int launch_cluster_update(const ClusterLaunch& l, cudaStream_t stream);   // mu (and prep) from perm, offsets
 int launch_permute_rows(const void* x, const int32_t* perm, int BH, int N, int D, bool inverse, void* out, int* status,
