@@ -320,58 +320,75 @@ __global__ void __launch_bounds__(kAsgThreads, 1)
   }
 }
 
-// Stable counting sort of one head's labels, one warp per (batch, head):
-// histogram in shared memory, an exclusive scan into the offsets (and the
-// offsets of the non-empty clusters: the query groups), then the rows in
-// ascending order, 32 at a time: lanes with equal labels rank themselves by
-// lane order (__match_any_sync) and the lowest of them moves the cluster's
-// cursor.  Labels are read 32 x kSortBatch at a time, a batch ahead of the
-// one being processed, so that their loads are in flight together.  A label
-// outside [0, C) is skipped and sets the device-check status (its row then
-// has no place in perm).
-constexpr int kSortBatch = 16;
+// Stable counting sort of one head's labels, one CTA of W warps per (batch,
+// head); warp w owns the contiguous rows [w seg, (w+1) seg):
+//   count  each warp counts its rows into its own histogram row hist[w][c];
+//   scan   per cluster, the column prefix over the warps gives each warp's
+//          first position inside the cluster, and a block-wide exclusive
+//          scan of the cluster totals gives the offsets (and the offsets of
+//          the non-empty clusters: the query groups);
+//   place  each warp walks its rows in ascending order, 32 at a time: lanes
+//          with equal labels rank themselves by lane order
+//          (__match_any_sync) and the lowest of them moves the warp's cursor.
+// Rows keep their order inside a cluster because the warps' segments are
+// ordered and each warp places its rows in order.  Labels are read
+// 32 x kSortBatch at a time, a batch ahead of the one being processed.  A
+// label outside [0, C) is skipped and sets the device-check status (its row
+// then has no place in perm).
+constexpr int kSortBatch = 8;
+constexpr int kSortMaxWarps = 16;
 
-__global__ void __launch_bounds__(32) cluster_sort_kernel(ClusterLaunch l, int* status) {
-  extern __shared__ __align__(16) int32_t cur[];  // [C]: counts, then cursors
-  const int lane = threadIdx.x;
+__global__ void __launch_bounds__(kSortMaxWarps * 32) cluster_sort_kernel(ClusterLaunch l, int* status) {
+  extern __shared__ __align__(16) int32_t hist[];  // [W][C]: counts, then cursors
+  __shared__ int32_t red_rows[kSortMaxWarps], red_ne[kSortMaxWarps];
+  __shared__ int bad_any;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, W = blockDim.x >> 5;
   const int64_t bh = blockIdx.x;
   const int N = l.N, C = l.C;
   const int32_t* lab = l.labels + bh * N;
-  for (int c = lane; c < C; c += 32) cur[c] = 0;
+  const int seg = (N + W - 1) / W;
+  const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
+  int32_t* my = hist + static_cast<int64_t>(warp) * C;
+  if (tid == 0) bad_any = 0;
+  for (int c = lane; c < C; c += 32) my[c] = 0;
   __syncwarp();
-  // labels of rows base + 32 k + lane, k < kSortBatch (-1 past N); the next
-  // batch's loads are issued before the current batch is processed
   auto load_batch = [&](int base, int (&v)[kSortBatch]) {
 #pragma unroll
     for (int k = 0; k < kSortBatch; ++k) {
       const int r = base + 32 * k + lane;
-      v[k] = r < N ? lab[r] : -1;
+      v[k] = r < s1 ? lab[r] : -1;
     }
   };
+  constexpr int kStep = 32 * kSortBatch;
   bool bad = false;
   int v[kSortBatch], nx[kSortBatch];
-  load_batch(0, v);
-  for (int base = 0; base < N; base += 32 * kSortBatch) {
-    if (base + 32 * kSortBatch < N) load_batch(base + 32 * kSortBatch, nx);
+  load_batch(s0, v);
+  for (int base = s0; base < s1; base += kStep) {
+    if (base + kStep < s1) load_batch(base + kStep, nx);
 #pragma unroll
     for (int k = 0; k < kSortBatch; ++k) {
       if (v[k] >= 0 && v[k] < C) {
-        atomicAdd(&cur[v[k]], 1);
-      } else if (base + 32 * k + lane < N) {
+        atomicAdd(&my[v[k]], 1);
+      } else if (base + 32 * k + lane < s1) {
         bad = true;
       }
     }
 #pragma unroll
     for (int k = 0; k < kSortBatch; ++k) v[k] = nx[k];
   }
-  __syncwarp();
-  // lane owns clusters [c0, c1)
-  const int E = (C + 31) / 32;
-  const int c0 = min(C, lane * E), c1 = min(C, c0 + E);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) bad_any = 1;
+  __syncthreads();
+
+  // scan: thread t owns clusters [c0, c1)
+  const int T = blockDim.x;
+  const int E = (C + T - 1) / T;
+  const int c0 = min(C, tid * E), c1 = min(C, c0 + E);
   int rows_local = 0, ne_local = 0;
   for (int c = c0; c < c1; ++c) {
-    rows_local += cur[c];
-    ne_local += cur[c] > 0 ? 1 : 0;
+    int n = 0;
+    for (int w = 0; w < W; ++w) n += hist[static_cast<int64_t>(w) * C + c];
+    rows_local += n;
+    ne_local += n > 0 ? 1 : 0;
   }
   int rows_incl = rows_local, ne_incl = ne_local;
 #pragma unroll
@@ -383,49 +400,71 @@ __global__ void __launch_bounds__(32) cluster_sort_kernel(ClusterLaunch l, int* 
       ne_incl += t1;
     }
   }
-  int run = rows_incl - rows_local, g = ne_incl - ne_local;
+  if (lane == 31) {
+    red_rows[warp] = rows_incl;
+    red_ne[warp] = ne_incl;
+  }
+  __syncthreads();
+  int rows_before = 0, ne_before = 0, rows_all = 0, ne_all = 0;
+  for (int w = 0; w < W; ++w) {
+    if (w < warp) {
+      rows_before += red_rows[w];
+      ne_before += red_ne[w];
+    }
+    rows_all += red_rows[w];
+    ne_all += red_ne[w];
+  }
+  int run = rows_before + rows_incl - rows_local, g = ne_before + ne_incl - ne_local;
   int32_t* off = l.offsets + bh * (C + 1);
   int32_t* grp = l.groups ? l.groups + bh * (C + 1) : nullptr;
   for (int c = c0; c < c1; ++c) {
-    const int n = cur[c];
+    int col = run;
+    for (int w = 0; w < W; ++w) {
+      int32_t& h = hist[static_cast<int64_t>(w) * C + c];
+      const int x = h;
+      h = col;
+      col += x;
+    }
+    const int n = col - run;
     off[c] = run;
     if (grp && n > 0) grp[g++] = run;
-    cur[c] = run;
-    run += n;
+    run = col;
   }
-  if (lane == 31) {
-    off[C] = rows_incl;
-    if (grp) grp[ne_incl] = rows_incl;
-    if (l.n_groups) l.n_groups[bh] = ne_incl;
+  if (tid == 0) {
+    off[C] = rows_all;
+    if (grp) grp[ne_all] = rows_all;
+    if (l.n_groups) l.n_groups[bh] = ne_all;
   }
-  __syncwarp();
+  __syncthreads();
+
+  // place
   int32_t* pm = l.perm + bh * N;
-  load_batch(0, v);
-  for (int base = 0; base < N; base += 32 * kSortBatch) {
-    if (base + 32 * kSortBatch < N) load_batch(base + 32 * kSortBatch, nx);
+  load_batch(s0, v);
+  for (int base = s0; base < s1; base += kStep) {
+    if (base + kStep < s1) load_batch(base + kStep, nx);
 #pragma unroll
     for (int k = 0; k < kSortBatch; ++k) {
       const int c = (v[k] >= 0 && v[k] < C) ? v[k] : -1;
       const unsigned peers = __match_any_sync(0xffffffffu, c);
       const int rank = __popc(peers & ((1u << lane) - 1u));
-      const int pos = c >= 0 ? cur[c] + rank : 0;
+      const int pos = c >= 0 ? my[c] + rank : 0;
       __syncwarp();
       if (c >= 0) {
         pm[pos] = base + 32 * k + lane;
-        if (rank == 0) cur[c] += __popc(peers);
+        if (rank == 0) my[c] += __popc(peers);
       }
       __syncwarp();
     }
 #pragma unroll
     for (int k = 0; k < kSortBatch; ++k) v[k] = nx[k];
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(status, 0, kStatusDeviceCheck);
+  if (tid == 0 && bad_any) atomicCAS(status, 0, kStatusDeviceCheck);
 }
 
 // mu_c = mean of cluster c's rows in permutation order (fp32, a fixed order,
 // so the result does not depend on scheduling); an empty cluster keeps its
-// centroid.  One warp per centroid; the hi / lo / norm operands of the next
-// assignment are written too.
+// centroid.  One warp per centroid, 16 row loads in flight; the hi / lo /
+// norm operands of the next assignment are written too.
 template <int D>
 __global__ void __launch_bounds__(kPrepWarps * 32) cluster_update_kernel(ClusterLaunch l) {
   constexpr int PER = D / 32;
@@ -443,45 +482,38 @@ __global__ void __launch_bounds__(kPrepWarps * 32) cluster_update_kernel(Cluster
     float acc[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
-    auto add_row = [&](int r) {
-      const uint16_t* p = xb + static_cast<int64_t>(r) * D;
-      if constexpr (PER == 4) {
-        const uint2 w = *reinterpret_cast<const uint2*>(p);
-        acc[0] += bf16f(w.x & 0xFFFF);
-        acc[1] += bf16f(w.x >> 16);
-        acc[2] += bf16f(w.y & 0xFFFF);
-        acc[3] += bf16f(w.y >> 16);
-      } else {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
-        acc[0] += bf16f(w & 0xFFFF);
-        acc[1] += bf16f(w >> 16);
-      }
-    };
-    int i = s;
-    for (; i + 4 <= e; i += 4) {
-      // the four rows' loads are issued before the first add
-      const int ra = pm[i], rb = pm[i + 1], rc = pm[i + 2], rd = pm[i + 3];
-      if constexpr (PER == 4) {
-        const uint2 wa = *reinterpret_cast<const uint2*>(xb + static_cast<int64_t>(ra) * D);
-        const uint2 wb = *reinterpret_cast<const uint2*>(xb + static_cast<int64_t>(rb) * D);
-        const uint2 wc = *reinterpret_cast<const uint2*>(xb + static_cast<int64_t>(rc) * D);
-        const uint2 wd = *reinterpret_cast<const uint2*>(xb + static_cast<int64_t>(rd) * D);
-        const uint2 w4[4] = {wa, wb, wc, wd};
+    // 32 positions at a time: lane k loads perm[b0 + k], then the rows go
+    // 16 loads in flight at a time and are added in position order
+    constexpr int kU = 16;
+    for (int b0 = s; b0 < e; b0 += 32) {
+      const int n = min(32, e - b0);
+      const int my_r = lane < n ? pm[b0 + lane] : 0;
+      for (int k0 = 0; k0 < n; k0 += kU) {
+        float f[kU][PER];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          acc[0] += bf16f(w4[k].x & 0xFFFF);
-          acc[1] += bf16f(w4[k].x >> 16);
-          acc[2] += bf16f(w4[k].y & 0xFFFF);
-          acc[3] += bf16f(w4[k].y >> 16);
+        for (int u = 0; u < kU; ++u) {
+          const int r = __shfl_sync(0xffffffffu, my_r, (k0 + u) & 31);
+          const uint16_t* p = xb + static_cast<int64_t>(r) * D;
+          if constexpr (PER == 4) {
+            const uint2 w = k0 + u < n ? *reinterpret_cast<const uint2*>(p) : make_uint2(0u, 0u);
+            f[u][0] = bf16f(w.x & 0xFFFF);
+            f[u][1] = bf16f(w.x >> 16);
+            f[u][2] = bf16f(w.y & 0xFFFF);
+            f[u][3] = bf16f(w.y >> 16);
+          } else {
+            const uint32_t w = k0 + u < n ? *reinterpret_cast<const uint32_t*>(p) : 0u;
+            f[u][0] = bf16f(w & 0xFFFF);
+            f[u][1] = bf16f(w >> 16);
+          }
         }
-      } else {
-        add_row(ra);
-        add_row(rb);
-        add_row(rc);
-        add_row(rd);
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+          if (k0 + u < n) {
+#pragma unroll
+            for (int q = 0; q < PER; ++q) acc[q] += f[u][q];
+          }
       }
     }
-    for (; i < e; ++i) add_row(pm[i]);
     const float inv = 1.0f / static_cast<float>(e - s);
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
@@ -570,13 +602,16 @@ int launch_cluster_assign(const ClusterLaunch& l, int num_sms, uint64_t timeout_
 }
 
 int launch_cluster_sort(const ClusterLaunch& l, int* status, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(l.C) * 4;
+  // as many warps per head as keep the per-warp histograms within 64 KB
+  int W = 16384 / (l.C > 0 ? l.C : 1);
+  W = W < 1 ? 1 : (W > kSortMaxWarps ? kSortMaxWarps : W);
+  const size_t smem = static_cast<size_t>(W) * l.C * 4;
   if (smem > 48 * 1024) {
     const cudaError_t e =
-        cudaFuncSetAttribute(cluster_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        cudaFuncSetAttribute(cluster_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
     if (e != cudaSuccess) return static_cast<int>(e);
   }
-  cluster_sort_kernel<<<l.BH, 32, smem, stream>>>(l, status);
+  cluster_sort_kernel<<<l.BH, W * 32, smem, stream>>>(l, status);
   return static_cast<int>(cudaGetLastError());
 }
 
