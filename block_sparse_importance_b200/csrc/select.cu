@@ -324,9 +324,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
 // Warp-per-row variant for rows of at most 32 * VPL blocks: lane l holds the
 // contiguous blocks [l*VPL, (l+1)*VPL) in registers, so every scan is a local
 // prefix plus one warp shuffle scan and no block-wide barrier is needed.  The
-// exact set's threshold is found by a bitwise binary search on the keys (the
-// largest t with #{key >= t} >= n_exact).  Same integer arithmetic and same
-// results as select_kernel.
+// exact set's threshold (the n_exact-th largest key, i.e. the largest t with
+// #{key >= t} >= n_exact) comes from a 4-round radix select with a per-warp
+// shared-memory histogram.  Same integer arithmetic and same results as
+// select_kernel.
 constexpr int kWarpRowsPerCta = 8;
 
 __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
@@ -397,13 +398,54 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
   // ---- exact set: threshold t = largest key with #{key >= t} >= n_exact
   uint64_t ex = 0;  // bit v: block base+v is exact
   if (n_exact > 0) {
-    uint32_t t = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = t | (1u << bit);
-      uint32_t c = 0;
+    // t = the n_exact-th largest key, by a radix select over the key bytes
+    // from the top: a 256-bin histogram of the keys that match the prefix
+    // so far, and the bin holding the remaining rank (lane l owns bins
+    // 8l .. 8l+7, so the bins above a lane's are those of higher lanes)
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sm) + kWarpRowsPerCta * (32 * VPL + VPL) + warp * 256;
+    uint32_t t = 0, mask = 0, kk = static_cast<uint32_t>(n_exact);
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
 #pragma unroll
-      for (int v = 0; v < VPL; ++v) c += (v < nv && key[v] >= cand) ? 1u : 0u;
-      if (__reduce_add_sync(0xffffffffu, c) >= static_cast<uint32_t>(n_exact)) t = cand;
+      for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0u;
+      __syncwarp();
+#pragma unroll
+      for (int v = 0; v < VPL; ++v)
+        if (v < nv && (key[v] & mask) == t) atomicAdd(&hist[(key[v] >> shift) & 255u], 1u);
+      __syncwarp();
+      uint32_t cnt[8], local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cnt[i] = hist[lane * 8 + i];
+        local += cnt[i];
+      }
+      uint32_t suf = local;  // keys in the bins of lanes >= this one
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += x;
+      }
+      const uint32_t above = suf - local;
+      const bool here = above < kk && suf >= kk;
+      uint32_t sel = 0, rem = 0;
+      if (here) {
+        uint32_t acc = above;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+          if (rem == 0 && acc + cnt[i] >= kk) {
+            sel = 8 * lane + i;
+            rem = kk - acc;
+          }
+          acc += cnt[i];
+        }
+      }
+      const int src = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
+      sel = __shfl_sync(0xffffffffu, sel, src);
+      rem = __shfl_sync(0xffffffffu, rem, src);
+      t |= sel << shift;
+      mask |= 255u << shift;
+      kk = rem;
+      __syncwarp();  // every lane has read the histogram before it is cleared
     }
     uint32_t gt = 0, eq = 0;
 #pragma unroll
@@ -623,7 +665,7 @@ __global__ void __launch_bounds__(kSelThreads) top_p_count_kernel(const float* _
 template <int VPL>
 int launch_select_warp(const SelectLaunch& s, cudaStream_t stream) {
   const long long rows = static_cast<long long>(s.B) * s.H * s.G;
-  const size_t smem = static_cast<size_t>(kWarpRowsPerCta) * (32 * VPL + VPL) * 4;
+  const size_t smem = static_cast<size_t>(kWarpRowsPerCta) * (32 * VPL + VPL + 256) * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_warp_kernel<VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
