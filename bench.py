@@ -205,6 +205,50 @@ def cpu_oracle_sample(w, inp, target_s: float = 12.0):
                       % (n, G, w.name, dt)}
 
 
+def cpu_cluster_sample(x_head, n_clusters: int, rounds: int, target_s: float = 6.0):
+    """Time the oracle's token clustering (fp64) of the first rows of one head,
+    growing the sample until it takes about `target_s` seconds; the rate is in
+    the distance products' TFLOP/s (2 n C d per round)."""
+    import oracle
+    N, d = x_head.shape[-2], x_head.shape[-1]
+
+    def run(n):
+        t0 = time.perf_counter()
+        oracle.cluster_tokens(x_head[..., :n, :], min(n_clusters, n), rounds)
+        return time.perf_counter() - t0
+
+    n = min(N, 2048)
+    dt = run(n)
+    while dt < target_s / 4 and n < N:
+        n = min(N, max(n + 1, int(n * min(8.0, target_s / max(dt, 1e-3)))))
+        dt = run(n)
+    flops = 2.0 * n * min(n_clusters, n) * d * rounds
+    # the oracle parallelises over (batch, head): one head runs on one thread
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s (computed)", "cores": 1,
+            "kind": "oracle",
+            "sample": "head 0 of Q, first %d of %d tokens, %d clusters, %d rounds: oracle clustering (fp64), %.1f s"
+                      % (n, N, min(n_clusters, n), rounds, dt)}
+
+
+def cpu_top_p_sample(mass_np, p: float, S: int, seed: int, target_s: float = 3.0):
+    """Time the oracle's top-p selector on the first plan rows of head 0."""
+    import oracle
+    G = mass_np.shape[2]
+
+    def run(g):
+        t0 = time.perf_counter()
+        oracle.select_top_p(mass_np[:, :1, :g], p, S, seed)
+        return time.perf_counter() - t0
+
+    g = min(G, 16)
+    dt = run(g)
+    while dt < target_s / 4 and g < G:
+        g = min(G, max(g + 1, int(g * min(8.0, target_s / max(dt, 1e-3)))))
+        dt = run(g)
+    return {"value": g / dt, "unit": "plan rows/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "head 0, first %d of %d plan rows: oracle top-p selector, %.2f s" % (g, G, dt)}
+
+
 def reference_arm(args):
     """--impl reference: the fp64 oracle on the host cores, bounded samples."""
     rank = int(os.environ.get("RANK", "0"))
@@ -395,8 +439,11 @@ def main():
         stages["select_top_p"] = {"ms": tp_ms, "p": args.top_p, "bytes": tp_bytes,
                                   "gbs": tp_bytes / (tp_ms * 1e-3) / 1e9,
                                   "frac_hbm": tp_bytes / (tp_ms * 1e-3) / 1e9 / hbm,
+                                  "rows_per_s": B * H * G / (tp_ms * 1e-3),
                                   "n_exact_mean": float(ke.mean()), "n_exact_min": int(ke.min()),
                                   "n_exact_max": int(ke.max())}
+        if world == 1 and not args.no_cpu_baseline:
+            stages["select_top_p"]["cpu_baseline"] = cpu_top_p_sample(mass.cpu().numpy(), args.top_p, S, w.seed)
         del ne_rows
 
     # the permuted layout's build (token clustering of Q and K, then the row
@@ -429,6 +476,8 @@ def main():
         stages["cluster"] = {"ms": c_ms, "n_clusters": C_t, "rounds": it_t, "tflop": c_flops / 1e12,
                              "tflops": c_flops / (c_ms * 1e-3) / 1e12,
                              "what": "isa_cluster of Q and of K, then permute_rows of Q, K and V"}
+        if world == 1 and not args.no_cpu_baseline:
+            stages["cluster"]["cpu_baseline"] = cpu_cluster_sample(wl.bf16_bits(q[:, :1].cpu()), C_t, it_t)
         del qp, kp, vp, cws
 
     # end to end through the C ABI from pinned host buffers
