@@ -245,8 +245,18 @@ def cpu_top_p_sample(mass_np, p: float, S: int, seed: int, target_s: float = 3.0
     while dt < target_s / 4 and g < G:
         g = min(G, max(g + 1, int(g * min(8.0, target_s / max(dt, 1e-3)))))
         dt = run(g)
+    # a whole head that takes less than the target is repeated until it does
+    reps = 1
+    while dt * reps < target_s / 4:
+        reps *= 2
+    if reps > 1:
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            run(g)
+        dt = (time.perf_counter() - t0) / reps
     return {"value": g / dt, "unit": "plan rows/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "head 0, first %d of %d plan rows: oracle top-p selector, %.2f s" % (g, G, dt)}
+            "sample": "head 0, first %d of %d plan rows, %d repetitions: oracle top-p selector, %.2f s"
+                      % (g, G, reps, dt * reps)}
 
 
 def reference_arm(args):
