@@ -189,3 +189,14 @@ def test_permuted_flow_matches_unpermuted(isa):
     assert isa.context().sync_status() == isa.ISA_OK
     out = isa.permute_rows(out_p, rq["perm"], inverse=True)
     assert (out.float() - dense.float()).abs().max().item() <= cases.ATTN_MAX_ABS
+
+
+def test_cluster_arguments(isa):
+    # host-side checks: nothing is enqueued
+    x = torch.zeros(1, 1, 64, 128, dtype=torch.bfloat16, device="cuda")
+    for C, it in [(0, 1), (65, 1), (4, 0)]:
+        with pytest.raises(isa.IsaError):
+            isa.cluster(x, C, it)
+    with pytest.raises(isa.IsaError):
+        isa.permute_rows(x, torch.zeros(1, 1, 64, dtype=torch.int32, device="cuda"), out=x)
+    assert isa.context().sync_status() == isa.ISA_OK
