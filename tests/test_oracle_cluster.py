@@ -13,7 +13,9 @@ permutation it is parameterised by):
   * after enough rounds the result is a Lloyd fixed point (every label is
     its row's nearest centroid, every centroid its cluster's mean);
   * well-separated generated clusters whose initial rows fall in distinct
-    clusters are recovered exactly.
+    clusters are recovered exactly;
+  * a hand-worked one-round case fixes the initial rows (the reading's
+    floor(c N / C)) and the tie rule.
 """
 import numpy as np
 import pytest
@@ -136,6 +138,23 @@ def test_well_separated_clusters_are_recovered():
     assert not amb[0, 0]
     assert np.array_equal(lab[0, 0], truth)
     assert np.array_equal(off[0, 0], np.arange(C + 1) * per)
+
+
+def test_initial_centroids_are_rows_c_n_over_c():
+    # one round from the initial centroids: rows 0, 2 and 4 of six (floor(c 6 / 3)),
+    # worked by hand; the values are such that every other ordered choice of three
+    # initial rows gives other labels or other means after the round
+    x = np.array([[2.0], [9.0], [14.0], [17.0], [23.0], [38.0]])
+    lab, perm, off, mu, _ = oracle.cluster_tokens(bf16_bits(x)[None, None], 3, 1)
+    # centroids 2, 14, 23: 9 is 5 from 14 and 7 from 2; 17 is 3 from 14 and 6 from 23
+    assert list(lab[0, 0]) == [0, 1, 1, 1, 2, 2]
+    np.testing.assert_allclose(mu[0, 0, :, 0], [2.0, 40.0 / 3.0, 30.5], rtol=1e-15)
+    # a tie goes to the lower centroid: 16 is 2 from both 14 and 18
+    x = np.array([[14.0], [16.0], [18.0]])
+    lab, _, _, _, amb = oracle.cluster_tokens(bf16_bits(x)[None, None], 2, 1)  # rows 0 and 1 start
+    assert list(lab[0, 0]) == [0, 1, 1]
+    lab2, _ = oracle.cluster_assign(bf16_bits(np.array([[16.0]])), np.array([[14.0], [18.0]]))
+    assert list(lab2) == [0]
 
 
 def test_arguments():

@@ -10,6 +10,7 @@
     n_exact = k_e and n_sample = S - k_e, row by row, uniform included.
 """
 import math
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -18,13 +19,16 @@ import oracle
 
 
 def brute_k(m: np.ndarray, p: float, S: int) -> int:
+    """The fewest blocks, by descending mass, whose quantised sum reaches the
+    share p of the row's total, compared as exact rationals (fl(p * total)
+    is the product the reading rounds once in fp64)."""
     vals = [float(x) if (math.isfinite(float(x)) and float(x) > 0.0) else 0.0 for x in m]
     mmax = max(vals)
     q = [math.floor(v / mmax * 2147483648.0) if (v > 0.0 and mmax > 0.0) else 0 for v in vals]
-    target = math.ceil(p * float(sum(q)))
+    share = Fraction(p * float(sum(q)))
     order = sorted(range(len(vals)), key=lambda b: (-vals[b], b))
     k, cum = 0, 0
-    while cum < target and k < len(vals):
+    while Fraction(cum) < share and k < len(vals):
         cum += q[order[k]]
         k += 1
     return min(k, S)
@@ -56,6 +60,16 @@ def test_top_p_count_matches_brute_force(nK, S, p):
         k, bad = oracle.top_p_count(m, p, S)
         assert not bad
         assert k == brute_k(m, p, S)
+
+
+def test_top_p_count_at_a_fractional_share():
+    # two equal blocks, q = 2^31 each; p = 1/2 + 2^-33 puts the share at
+    # 2^31 + 1/2: one block falls short by half a unit, so both are needed
+    m = np.array([1.0, 1.0], np.float32)
+    p = 0.5 + 2.0 ** -33
+    assert p * 2.0 ** 32 == 2.0 ** 31 + 0.5
+    assert oracle.top_p_count(m, p, 2)[0] == 2 == brute_k(m, p, 2)
+    assert oracle.top_p_count(m, 0.5, 2)[0] == 1 == brute_k(m, 0.5, 2)
 
 
 def test_top_p_count_edges():
