@@ -36,19 +36,21 @@ def test_dense_limit_matches_library_attention():
     out, lse = oracle.dense_attention(q, k, v, scale, rows)
     want = np.stack([ref[h, r].numpy() for h, r in rows])
     assert np.max(np.abs(out - want)) < 1e-12
-    # all blocks exact, log_w = 0: the sparse pass is dense attention
-    Bk, Bq = 16, 64
-    off = np.minimum(np.arange(0, N + Bq, Bq), N).astype(np.int32)
-    G, nK = len(off) - 1, -(-N // Bk)
-    idx = np.tile(np.arange(nK, dtype=np.int32), (1, H, G, 1))
-    lw = np.zeros_like(idx, dtype=np.float32)
-    res = oracle.attention(q, k, v, off, Bk, idx, lw, scale, [(0, h, g) for h in range(H) for g in range(G)])
-    i = 0
-    for h in range(H):
-        for g in range(G):
-            o, l = res[i]
-            i += 1
-            assert np.max(np.abs(o - ref[h, off[g]:off[g + 1]].numpy())) < 1e-12
+    # all blocks exact, log_w = 0: the sparse pass is dense attention, with a
+    # partial last key block (16) and with blocks that divide N (20)
+    for Bk in (16, 20):
+        Bq = 64
+        off = np.minimum(np.arange(0, N + Bq, Bq), N).astype(np.int32)
+        G, nK = len(off) - 1, -(-N // Bk)
+        idx = np.tile(np.arange(nK, dtype=np.int32), (1, H, G, 1))
+        lw = np.zeros_like(idx, dtype=np.float32)
+        res = oracle.attention(q, k, v, off, Bk, idx, lw, scale, [(0, h, g) for h in range(H) for g in range(G)])
+        i = 0
+        for h in range(H):
+            for g in range(G):
+                o, l = res[i]
+                i += 1
+                assert np.max(np.abs(o - ref[h, off[g]:off[g + 1]].numpy())) < 1e-12
 
 
 def test_sparse_pass_matches_masked_library_attention():
