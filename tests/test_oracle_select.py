@@ -224,3 +224,17 @@ def test_edge_cases():
     assert bad and idx[0] == 2
     with pytest.raises(ValueError):
         oracle.select_row(m, 3, 2, 0)
+
+
+def test_non_positive_mass_counts_as_zero():
+    # a mass estimate carries no weight below zero: negative entries select exactly
+    # like zeros, for every split and uniform
+    rng = np.random.default_rng(12)
+    for _ in range(20):
+        m = rng.normal(0.0, 1.0, 40).astype(np.float32)
+        z = np.where(m > 0, m, 0.0).astype(np.float32)
+        for ne, ns in [(5, 10), (0, 12), (20, 20)]:
+            U = int(rng.integers(0, 2 ** 32))
+            a = oracle.select_row(m, ne, ns, U)
+            b = oracle.select_row(z, ne, ns, U)
+            assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]) and not a[3]
