@@ -341,7 +341,6 @@ constexpr int kSortMaxWarps = 16;
 __global__ void __launch_bounds__(kSortMaxWarps * 32) cluster_sort_kernel(ClusterLaunch l, int* status) {
   extern __shared__ __align__(16) int32_t hist[];  // [W][C]: counts, then cursors
   __shared__ int32_t red_rows[kSortMaxWarps], red_ne[kSortMaxWarps];
-  __shared__ int bad_any;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, W = blockDim.x >> 5;
   const int64_t bh = blockIdx.x;
   const int N = l.N, C = l.C;
@@ -349,7 +348,6 @@ __global__ void __launch_bounds__(kSortMaxWarps * 32) cluster_sort_kernel(Cluste
   const int seg = (N + W - 1) / W;
   const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
   int32_t* my = hist + static_cast<int64_t>(warp) * C;
-  if (tid == 0) bad_any = 0;
   for (int c = lane; c < C; c += 32) my[c] = 0;
   __syncwarp();
   auto load_batch = [&](int base, int (&v)[kSortBatch]) {
@@ -376,7 +374,7 @@ __global__ void __launch_bounds__(kSortMaxWarps * 32) cluster_sort_kernel(Cluste
 #pragma unroll
     for (int k = 0; k < kSortBatch; ++k) v[k] = nx[k];
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) bad_any = 1;
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(status, 0, kStatusDeviceCheck);
   __syncthreads();
 
   // scan: thread t owns clusters [c0, c1)
@@ -458,7 +456,6 @@ __global__ void __launch_bounds__(kSortMaxWarps * 32) cluster_sort_kernel(Cluste
 #pragma unroll
     for (int k = 0; k < kSortBatch; ++k) v[k] = nx[k];
   }
-  if (tid == 0 && bad_any) atomicCAS(status, 0, kStatusDeviceCheck);
 }
 
 // mu_c = mean of cluster c's rows in permutation order (fp32, a fixed order,
