@@ -99,3 +99,15 @@ def test_plan_flops_matches_brute_force():
                 valid = min(Bk, N - b * Bk)
                 want += 4.0 * d * valid * (offsets[g + 1] - offsets[g])
     assert bench.plan_flops(idx, offsets, N, Bk, d) == want
+
+
+def test_oracle_samples_of_the_widening_stages():
+    # the CPU baselines of the layout build and the top-p stage: bounded samples of
+    # the oracle, reported with the threads they used
+    rng = np.random.default_rng(0)
+    x = (rng.normal(size=(1, 1, 600, 64)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    c = bench.cpu_cluster_sample(x, 16, 2, target_s=0.2)
+    assert c["kind"] == "oracle" and c["cores"] == 1 and c["value"] > 0 and "600 tokens" in c["sample"]
+    m = np.exp(rng.normal(size=(1, 2, 30, 100))).astype(np.float32)
+    t = bench.cpu_top_p_sample(m, 0.5, 12, 0, target_s=0.2)
+    assert t["kind"] == "oracle" and t["unit"] == "plan rows/s" and t["value"] > 0 and "30 of 30" in t["sample"]
