@@ -11,7 +11,7 @@
 //   assign  argmin_c ||x - mu_c||^2 = argmin_c (|mu_c|^2 - 2 x.mu_c), ties to
 //           the lower c; the dot products run on the tensor cores (tcgen05,
 //           fp32 accumulators in TMEM) with x exact in bf16 and mu split into
-//           bf16 hi + lo parts (relative error 2^-16), two products per k-step;
+//           bf16 hi + lo parts (relative error at most 2^-18), two products per k-step;
 //   sort    a stable counting sort of the labels: perm lists the rows in
 //           (label, row) order, offsets[c] .. offsets[c + 1] are cluster c's;
 //   update  mu_c = the fp32 mean of cluster c's rows taken in permutation

@@ -79,11 +79,10 @@ __global__ void __launch_bounds__(kScoreThreads) key_means_kernel(const uint16_t
   }
 }
 
-// ---------------------------------------------------------------- k-means
-// One CTA (8 warps) per (batch*head, group).  Rows stream through shared
-// memory 128 at a time (a group of <= 128 rows is loaded once), rows padded to
-// D + 8 elements so that ldmatrix reads are free of bank conflicts.
 // ---------------------------------------------- k-means, one warp per group
+// Rows stream through the warp's shared-memory buffer 128 at a time (a group
+// of <= 128 rows is loaded once), padded to D + 8 elements so that ldmatrix
+// reads are free of bank conflicts.
 // Assignment: dist_c = |mu_c|^2 - 2 x.mu_c (|x|^2 is common to all c) with the
 // dots on tensor cores: x is exact in bf16 and mu_c is split into bf16
 // hi + lo parts (relative error 2^-18), two mma.sync per 16x8x16 tile.

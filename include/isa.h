@@ -206,7 +206,7 @@ ISA_API isa_status isa_select_top_p(isa_context* ctx, const isa_shape* shape, co
  * inverse = 1); keys permuted by their own clustering form the key blocks.
  * Only batch, heads, seq_len and head_dim of `shape` are read; x is
  * [B,H,N,d] bf16.  The distances use x exact in bf16 and mu split into bf16
- * hi + lo parts (relative error 2^-16), so an assignment decided by a margin
+ * hi + lo parts (relative error at most 2^-18), so an assignment decided by a margin
  * below ~3e-5 of ||x||^2 + ||mu||^2 may differ from an exact computation.
  * ------------------------------------------------------------------------- */
 /* Scratch for isa_cluster / isa_cluster_assign / isa_cluster_update: the
