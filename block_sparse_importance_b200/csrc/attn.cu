@@ -697,11 +697,9 @@ int launch_d(const AttnLaunch& l, const void* q, const void* k, const void* v, c
   }
   const long long pairs = (static_cast<long long>(BH) * tiles_upper + 1) / 2;
   const int grid = static_cast<int>(pairs < l.num_sms ? pairs : l.num_sms);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
+  {
+    const cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(attn_kernel<D>), Lay::kAlloc);
     if (e != cudaSuccess) return static_cast<int>(e);
-    attr_set = true;
   }
   attn_kernel<D><<<grid, kThreads, Lay::kAlloc, stream>>>(tq, tk, tv, a);
   return static_cast<int>(cudaGetLastError());

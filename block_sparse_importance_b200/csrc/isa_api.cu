@@ -722,6 +722,34 @@ isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, const isa
 
 }  // extern "C"
 
+namespace isa_impl {
+
+cudaError_t ensure_smem_attr(const void* func, int bytes) {
+  struct Entry {
+    const void* func;
+    int device, bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& x : done)
+    if (x.func == func && x.device == dev && x.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  for (Entry& x : done)
+    if (x.func == func && x.device == dev) {
+      x.bytes = bytes;
+      return cudaSuccess;
+    }
+  done.push_back({func, dev, bytes});
+  return cudaSuccess;
+}
+
+}  // namespace isa_impl
+
 // ---------------------------------------------------------------------------
 // isa_attention_noalloc: isa_attention for callers that cannot allocate.
 //
@@ -738,7 +766,8 @@ isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, const isa
 // a host-side stand-in, so the device address is looked up with
 // cudaGetSymbolAddress the first time the entry point runs on a device (with
 // that device current) and cached per device.  Make that first call on each
-// device before any stream capture.  Every call shares the one array and it
+// device before any stream capture.  A device reset may move the array and
+// leave the cached address stale, so the entry point is not for use after one.  Every call shares the one array and it
 // keeps the last call's contents; the tile-list kernel rewrites every entry it
 // uses (and the count) on each call, so nothing needs clearing.  Calls whose
 // kernels overlap on the GPU (different streams, no ordering between them)

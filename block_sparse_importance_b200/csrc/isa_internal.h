@@ -15,6 +15,12 @@ enum : int { kStatusOk = 0, kStatusTimeout = 4, kStatusDeviceCheck = 5 };
 // Per-wait time limit of every bounded pipeline wait in the kernels.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 
+// Opts `func` into `bytes` of dynamic shared memory on the current device.
+// The attribute belongs to the function in the current device's context, so a
+// process that drives several GPUs needs it once per (function, device); the
+// record of what has been set is kept under a mutex.
+cudaError_t ensure_smem_attr(const void* func, int bytes);
+
 // ------------------------------------------------------------- attention
 enum AttnMode : int {
   kAttnGroups = 0,  // uniform query groups of <= 128 rows: one tile per group

@@ -697,12 +697,9 @@ int launch_mass(const ScoreLaunch& s, int nK, int BH, cudaStream_t stream) {
   using L = MassLayout<D>;
   CUtensorMap thi, tlo;
   if (!make_bf16_map(&thi, s.kbar_hi, BH, nK, D, 128) || !make_bf16_map(&tlo, s.kbar_lo, BH, nK, D, 128)) return -1;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(mass_kernel<D, Cp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(L::kAlloc));
+  {
+    const cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(mass_kernel<D, Cp>), static_cast<int>(L::kAlloc));
     if (e != cudaSuccess) return static_cast<int>(e);
-    attr = true;
   }
   constexpr int gpt = 128 / Cp;
   mass_kernel<D, Cp><<<dim3((s.G + gpt - 1) / gpt, BH), kMassThreads, L::kAlloc, stream>>>(
@@ -719,22 +716,18 @@ int launch_score_d(const ScoreLaunch& s, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
   using KL = KmLayout<D>;
-  static int km_blocks_per_sm[2] = {0, 0};
-  if (!km_blocks_per_sm[0]) {
-    e = cudaFuncSetAttribute(kmeans_warp_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(KL::kAlloc));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(kmeans_warp_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(KL::kAlloc));
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&km_blocks_per_sm[0], kmeans_warp_kernel<D, 1>,
-                                                        kKmWarps * 32, KL::kAlloc);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&km_blocks_per_sm[1], kmeans_warp_kernel<D, 2>,
-                                                        kKmWarps * 32, KL::kAlloc);
-    if (e != cudaSuccess) return static_cast<int>(e);
-    if (km_blocks_per_sm[0] < 1 || km_blocks_per_sm[1] < 1) return static_cast<int>(cudaErrorInvalidConfiguration);
-  }
+  int km_blocks_per_sm[2] = {0, 0};
+  e = ensure_smem_attr(reinterpret_cast<const void*>(kmeans_warp_kernel<D, 1>), static_cast<int>(KL::kAlloc));
+  if (e == cudaSuccess)
+    e = ensure_smem_attr(reinterpret_cast<const void*>(kmeans_warp_kernel<D, 2>), static_cast<int>(KL::kAlloc));
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&km_blocks_per_sm[0], kmeans_warp_kernel<D, 1>, kKmWarps * 32,
+                                                      KL::kAlloc);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&km_blocks_per_sm[1], kmeans_warp_kernel<D, 2>, kKmWarps * 32,
+                                                      KL::kAlloc);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  if (km_blocks_per_sm[0] < 1 || km_blocks_per_sm[1] < 1) return static_cast<int>(cudaErrorInvalidConfiguration);
   {
     // a persistent grid: every warp walks groups with a stride of the grid's warps
     const long long items = static_cast<long long>(BH) * s.G;

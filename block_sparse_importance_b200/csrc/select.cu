@@ -667,8 +667,7 @@ int launch_select_warp(const SelectLaunch& s, cudaStream_t stream) {
   const long long rows = static_cast<long long>(s.B) * s.H * s.G;
   const size_t smem = static_cast<size_t>(kWarpRowsPerCta) * (32 * VPL + VPL + 256) * 4;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(select_warp_kernel<VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_warp_kernel<VPL>), static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
   }
   const unsigned grid = static_cast<unsigned>((rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta);
@@ -682,8 +681,7 @@ int launch_top_p_count(const float* mass, int rows, int nK, double top_p, int S,
                        cudaStream_t stream) {
   const size_t smem = static_cast<size_t>(nK) * 8 + 16;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(top_p_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(top_p_count_kernel), static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
   }
   top_p_count_kernel<<<static_cast<unsigned>(rows), kSelThreads, smem, stream>>>(mass, nK, top_p, S, ne_rows, status);
@@ -697,8 +695,7 @@ int launch_select(const SelectLaunch& s, cudaStream_t stream) {
   if (s.nK <= 32 * 64) return launch_select_warp<64>(s, stream);
   const size_t smem = static_cast<size_t>(s.nK) * 9 + 16;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel), static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
   }
   const long long rows = static_cast<long long>(s.B) * s.H * s.G;

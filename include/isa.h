@@ -206,8 +206,12 @@ ISA_API isa_status isa_select_top_p(isa_context* ctx, const isa_shape* shape, co
  * inverse = 1); keys permuted by their own clustering form the key blocks.
  * Only batch, heads, seq_len and head_dim of `shape` are read; x is
  * [B,H,N,d] bf16.  The distances use x exact in bf16 and mu split into bf16
- * hi + lo parts (relative error at most 2^-18), so an assignment decided by a margin
- * below ~3e-5 of ||x||^2 + ||mu||^2 may differ from an exact computation.
+ * hi + lo parts (relative error at most 2^-18).  Relative to ||x||^2 + ||mu||^2,
+ * the split moves a distance by at most 2^-18 (4e-6), and the fp32
+ * accumulation of the d-term dot product and of ||mu||^2 by at most about
+ * 2 d 2^-24 (1.5e-5 at d = 128): below 2e-5 together.  An assignment decided
+ * by a margin below 3e-5 of that scale may therefore differ from an exact
+ * computation (the bound is deliberately loose).
  * ------------------------------------------------------------------------- */
 /* Scratch for isa_cluster / isa_cluster_assign / isa_cluster_update: the
  * centroids' bf16 hi / lo parts and squared norms (C rounded up to 64).
@@ -276,9 +280,11 @@ ISA_API isa_status isa_attention(isa_context* ctx, const isa_shape* shape, const
 
 /* ---------------------------------------------------------------------------
  * isa_dense_attention -- the 100%-density limit: softmax(scale Q K^T) V over
- * all keys, by the same tensor-core kernel with the whole sequence as plan
- * and zero log-weights.  Groups are ignored.  q, k, v, out as in
- * isa_attention; lse optional.
+ * all keys ("AB-Attention", problem statement: full attention weighs every
+ * query against every key, which the sparse pass estimates; with every block
+ * in the exact set the sparse pass reduces to this).  The same tensor-core
+ * kernel runs with the whole sequence as plan and zero log-weights.  Groups
+ * are ignored.  q, k, v, out as in isa_attention; lse optional.
  * ------------------------------------------------------------------------- */
 ISA_API isa_status isa_dense_attention(isa_context* ctx, const isa_shape* shape, const void* q,
                                const void* k, const void* v, void* out, float* lse, void* stream);
@@ -310,7 +316,10 @@ ISA_API isa_status isa_pipeline(isa_context* ctx, const isa_shape* shape, const 
  * Returns after enqueueing; `stream` completes only after the last output
  * copy, so out_host is valid once `stream` is synchronised.  Work already on
  * `stream` is finished before the arena is overwritten.  Calls that share a
- * context share its copy streams.
+ * context share its copy streams.  Unlike the other calls this one creates
+ * CUDA objects: its first call on a context creates the two copy streams
+ * (kept until isa_destroy), and every call creates and releases a few
+ * events.  It is therefore not meant for stream capture into a CUDA graph.
  * ------------------------------------------------------------------------- */
 ISA_API size_t isa_pipeline_host_workspace_bytes(const isa_shape* shape, const isa_params* params);
 ISA_API isa_status isa_pipeline_host(isa_context* ctx, const isa_shape* shape, const isa_params* params,
@@ -346,9 +355,11 @@ ISA_API isa_status isa_debug_set(isa_context* ctx, int32_t knob, uint64_t value)
  * (larger shapes return ISA_ERR_INVALID_ARG).  Every GPU that loads the
  * library holds that 1 MiB until the process exits.  The first call on each
  * device looks up the array's device address (make that first call before
- * any stream capture).  All calls share the one array: calls whose kernels
- * overlap on the GPU race on it, so order them (one stream, or events).  The
- * call allocates nothing.
+ * any stream capture) and keeps it for the life of the process; a device
+ * reset (cudaDeviceReset, or a reset of the primary context) may move the
+ * array, so do not call this entry point after one.  All calls share the one
+ * array: calls whose kernels overlap on the GPU race on it, so order them
+ * (one stream, or events).  The call allocates nothing.
  * ------------------------------------------------------------------------- */
 ISA_API isa_status isa_attention_noalloc(isa_context* ctx, const isa_shape* shape, const void* q,
                                          const void* k, const void* v, const int32_t* idx,

@@ -111,3 +111,14 @@ def test_oracle_samples_of_the_widening_stages():
     m = np.exp(rng.normal(size=(1, 2, 30, 100))).astype(np.float32)
     t = bench.cpu_top_p_sample(m, 0.5, 12, 0, target_s=0.2)
     assert t["kind"] == "oracle" and t["unit"] == "plan rows/s" and t["value"] > 0 and "30 of 30" in t["sample"]
+
+
+def test_roofline_peak_choice():
+    import bench
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    # a short timed region is held against the burst figure
+    assert bench.roofline_peak(peaks, 300.0, {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0}) == (1600.0, "burst")
+    # a long one at full clock too; a long one below it against the sustained figure
+    assert bench.roofline_peak(peaks, 5000.0, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}) == (1600.0, "burst")
+    assert bench.roofline_peak(peaks, 5000.0, {"sm_mhz": 1400.0, "sm_max_mhz": 1965.0}) == (1400.0, "sustained")
+    assert bench.roofline_peak(peaks, 5000.0, None) == (1400.0, "sustained")

@@ -30,7 +30,7 @@ def isa():
     return m
 
 
-@pytest.mark.parametrize("name", ["wan13", "wan14_10", "hunyuan", "varclust"])
+@pytest.mark.parametrize("name", ["wan13", "wan14_5", "wan14_10", "wan14_20", "hunyuan", "varclust"])
 def test_full_layer(isa, name):
     w = wl.preset(name)
     inp = wl.make_inputs(w, "cuda")
@@ -65,7 +65,11 @@ def test_full_layer(isa, name):
     # scorer
     m_ref, _, _, amb = oracle.score(qb, kb, off, w.k_block, w.n_clusters, w.n_iters, w.scale)
     ok = ~amb
-    assert ok.mean() > 0.5
+    # share of groups whose fp64 clustering met no near tie: about 0.93-0.96
+    # on the presets with uniform 128-row groups; varclust's clusters hold up
+    # to 1024 rows drawn around a single centre, where near ties are common
+    # (about 0.68 measured on seeded heads)
+    assert ok.mean() >= (0.6 if w.variable_groups else 0.85)
     r = cases.rel_l2(m_all[:, heads][ok], m_ref[ok])
     assert r <= cases.MASS_REL_L2, r
 
@@ -103,3 +107,40 @@ def test_full_layer(isa, name):
     ref = np.concatenate(ref)
     assert cases.rel_l2(got, ref) <= cases.ATTN_REL_L2
     assert np.abs(got - ref).max() <= cases.ATTN_MAX_ABS
+
+
+@pytest.mark.parametrize("name", ["wan14_10", "hunyuan"])
+def test_dense_limit_full_length(isa, name):
+    """isa_dense_attention over the whole layer at the preset's sequence
+    length (75 600 / 118 800 keys per row, as the benchmark runs it), against
+    the oracle's dense softmax attention on sampled rows of the first and last
+    head: max abs <= 5e-3 on the output, lse within 1e-2.  The sample includes
+    every row of the ragged last 128-row query tile."""
+    w = wl.preset(name)
+    inp = wl.make_inputs(w, "cuda")
+    q, k, v = inp.q, inp.k, inp.v
+    B, H, N, d = q.shape
+    lay = isa.layout_for(q, w.k_block, w.q_block, scale=w.scale)
+    out, lse = isa.dense_attention(q, k, v, lay, want_lse=True)
+    assert isa.context().sync_status() == isa.ISA_OK
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+    heads = [0, H - 1]
+    tail0 = (N - 1) // 128 * 128                         # first row of the last query tile
+    rng = np.random.default_rng(11)
+    rows = []
+    for j in range(len(heads)):
+        body = np.sort(rng.choice(tail0, 256 - (N - tail0), replace=False))
+        rows += [(j, int(r)) for r in body] + [(j, r) for r in range(tail0, N)]
+    qb = wl.bf16_bits(q[:, heads])
+    kb = wl.bf16_bits(k[:, heads])
+    vb = wl.bf16_bits(v[:, heads])
+    ref, ref_lse = oracle.dense_attention(qb, kb, vb, w.scale, rows)
+    o_h = out[0, heads].float().cpu().numpy()
+    l_h = lse[0, heads].cpu().numpy()
+    jj = np.array([j for j, _ in rows])
+    rr = np.array([r for _, r in rows])
+    got = o_h[jj, rr].astype(np.float64)
+    got_lse = l_h[jj, rr].astype(np.float64)
+    assert np.abs(got - ref).max() <= cases.DENSE_MAX_ABS
+    assert np.abs(got_lse - ref_lse).max() < 1e-2

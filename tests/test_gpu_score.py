@@ -34,7 +34,7 @@ def _run(isa, c: Case):
     assert np.all(cnt.sum(-1) == sizes[None, None, :])                 # valid everywhere
     assert np.allclose(mass.sum(-1), sizes[None, None, :], rtol=1e-4)  # sum_b m = n_g
     ok = ~amb
-    assert ok.mean() > 0.5
+    assert ok.mean() >= 0.85
     assert np.array_equal(cnt[ok], cnt_ref[ok])
     live = (cnt_ref > 0)[..., None] & ok[..., None, None]
     diff = np.abs(cen - cen_ref)
@@ -57,6 +57,6 @@ def test_score_matches_oracle(isa, preset, N, Bk, Bq, C):
 
 
 def test_score_variable_clusters(isa):
-    off = cases.random_offsets(2000, 16, 600, seed=5)
-    c = Case("wan13", 2, 2000, 64, 128, 2, 2, offsets=off)
+    off = cases.random_offsets(4000, 16, 300, seed=5)     # 30 clusters, some above one tile
+    c = Case("wan13", 2, 4000, 64, 128, 2, 2, offsets=off)
     _run(isa, c)
