@@ -274,12 +274,14 @@ def cpu_top_p_sample(mass_np, p: float, S: int, seed: int, target_s: float = 3.0
                       % (g, G, reps, dt * reps)}
 
 
-def time_plan_reuse(isa, ctx, stream, w, lay, q, k, v, mass, idx, lw, out, sws, aws, rs=(1, 2, 4, 8), cycles=2):
+def time_plan_reuse(isa, ctx, stream, w, lay, q, k, v, mass, idx, lw, out, sws, aws, rs=(1, 2, 4, 8), calls=8):
     """ms per attention call when one plan serves r calls, measured: each cycle
     runs isa_score and isa_select once on the current activations and then r
     isa_attention calls, alternating between the activations and a perturbed
     copy (x + 0.05 N(0, 1), in bf16), as consecutive denoising steps would
-    present them.  Events bracket the whole loop of `cycles` cycles."""
+    present them.  Every r runs the same number of attention calls (`calls`,
+    calls / r cycles) after the same idle pause, so that each loop meets the
+    GPU at the same clock and power state; events bracket the loop."""
     import torch
     gen = torch.Generator(device=q.device)
     gen.manual_seed(1234)
@@ -296,6 +298,9 @@ def time_plan_reuse(isa, ctx, stream, w, lay, q, k, v, mass, idx, lw, out, sws, 
                 qa, ka, va = alt[j % 2]
                 isa.attention(qa, ka, va, idx, lw, lay, out=out, workspace=aws, ctx=ctx)
         cycle()
+        torch.cuda.synchronize()
+        time.sleep(0.5)
+        cycles = max(1, calls // r)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(cycles):

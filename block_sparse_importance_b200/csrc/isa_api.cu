@@ -231,6 +231,7 @@ isa_status do_select(isa_context* ctx, const isa_shape* s, const float* mass, in
   l.log_w = log_w;
   l.ne_rows = ne_rows;
   l.status = ctx->d_status;
+  l.num_sms = ctx->num_sms;
   return cuda_status(ctx, launch_select(l, st), "isa_select");
 }
 

@@ -62,6 +62,7 @@ struct SelectLaunch {
   // it, n_exact + n_sample is the plan size and row r uses ne_rows[r] exact
   const int32_t* ne_rows;
   int* status;
+  int num_sms;
 };
 int launch_select(const SelectLaunch& s, cudaStream_t stream);
 // Exact-set sizes under the top-p rule, one per plan row, into ne_rows.

@@ -113,7 +113,8 @@ __global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16
                                                                     int G, int q_block,
                                                                     const int32_t* __restrict__ off, int C,
                                                                     int iters, float* __restrict__ centroids,
-                                                                    int32_t* __restrict__ counts, int* status) {
+                                                                    int32_t* __restrict__ counts, int min_rows,
+                                                                    int* status) {
   using namespace isa_dev;
   using L = KmLayout<D>;
   constexpr int XS = L::XS;
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16
       r1 = min(N, r0 + q_block);
     }
     const int n = r1 - r0;
+    if (n <= min_rows) continue;  // the tensor-core kernel runs the groups of at most min_rows rows
     const uint16_t* qg = q + (bh * N + r0) * D;
     // rows [cs, cs + rc) of the group into the warp's buffer (zero past rc),
     // with the column of ones beside each valid row
@@ -352,6 +354,439 @@ __global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16
   }
 }
 
+
+// --------------------------------------- k-means on tcgen05 (d = 128)
+// Groups of at most 128 rows.  A persistent CTA per SM streams the groups'
+// 128-row Q tiles through a ring of kKtSlots shared-memory buffers (TMA,
+// 128-byte swizzle), and kKtSets sets of four warps each run one group's
+// k-means at a time, every round on the tile in shared memory:
+//   assign  S = X [hi | lo]^T (M = 128 rows, N = 2 C', K = d; the set writes
+//           the centroids' bf16 hi and lo parts as an MN-major operand); one
+//           thread per row (TMEM lane) takes argmin_c |mu_c|^2 - 2 (S_hi,c +
+//           S_lo,c), ties to the lower c, and writes its row of the one-hot
+//           matrix OH (MN-major: 128 rows x 16 cluster slots);
+//   update  Sum^T = X^T OH (M = d dimensions, N = 16, K = 128 rows; the same
+//           X tile read MN-major); one thread per dimension (TMEM lane)
+//           multiplies its row of Sum^T by the reciprocal counts (ballots of
+//           the labels); an empty cluster keeps its centroid.
+// Thread t of a set keeps mu_c[t] for every c in registers across rounds.  A
+// set issues its own MMAs (one elected lane of its first warp) and waits for
+// them on its own barrier, so one set's waits overlap the other sets' work.
+// The operands a set writes (centroid parts, one-hot rows) are 16-byte rows
+// of the no-swizzle MN-major layout: 8 consecutive N entries of one K index
+// per 16 bytes, so each thread stores whole vectors.
+// Warp 4 kKtSets is the TMA producer.  Every wait is bounded.
+constexpr int kKtSets = 4;
+constexpr int kKtSlots = 5;
+constexpr int kKtThreads = (4 * kKtSets + 1) * 32;
+
+template <int CP>
+struct KtLayout {
+  static constexpr uint32_t kXBytes = 128 * 128 * 2;  // 128 rows x 128 dims, two 64-dim boxes
+  static constexpr uint32_t kBox = 128 * 128;
+  static constexpr uint32_t kX = 0;
+  // MN-major no-swizzle operands: the 8-entry N group j of K index k at
+  // j * kNGroup + k * 16 (K groups of 8 packed at 128-byte steps)
+  static constexpr uint32_t kNGroup = 128 * 16;
+  static constexpr uint32_t kMcBytes = (2 * CP / 8) * kNGroup;  // hi groups, then lo groups
+  static constexpr uint32_t kOhBytes = 2 * kNGroup;             // 16 cluster slots
+  static constexpr uint32_t kMc = kKtSlots * kXBytes;
+  static constexpr uint32_t kOh = kMc + kKtSets * kMcBytes;
+  // per set: |mu|^2 partials [16][4], |mu|^2 [16], counts [16], reciprocal counts [16]
+  static constexpr uint32_t kRed = kOh + kKtSets * kOhBytes;
+  static constexpr uint32_t kRedBytes = (64 + 16 + 16 + 16) * 4;
+  static constexpr uint32_t kBar = kRed + kKtSets * kRedBytes;
+  static constexpr int kXFull = 0, kXEmpty = kKtSlots, kMmaDone = 2 * kKtSlots, kNumBars = 2 * kKtSlots + kKtSets;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // TMEM address, abort flag; released[] at +16
+  static constexpr uint32_t kAlloc = kMisc + 16 + 4 * kKtSlots + 1024;
+};
+
+// Byte offset of element (row r, column c) in a K-major 128-byte-swizzled
+// tile of `rows` rows whose columns come in 64-element chunks.
+__device__ __forceinline__ uint32_t sw128_off(int rows, int r, int c) {
+  return static_cast<uint32_t>((c >> 6) * rows * 128 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2);
+}
+
+// Sums v[0 .. CP) over the warp's lanes: lane l ends with the total of
+// element e(l) = sum over the halving steps of (lane bit set) * (half size).
+template <int CP>
+__device__ __forceinline__ float warp_sum_scatter(float (&v)[CP], int lane, int& elem) {
+  int base = 0;
+#pragma unroll
+  for (int half = CP / 2, o = 16; half >= 1; half >>= 1, o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < half; ++j) {
+      const float send = up ? v[j] : v[j + half];
+      const float keep = up ? v[j + half] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+    base += up ? half : 0;
+  }
+  float r = v[0];
+  // the lane bits the halving steps did not use
+#pragma unroll
+  for (int o = 32 / CP / 2; o >= 1; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+  elem = base;
+  return r;
+}
+
+template <int CP>
+__global__ void __launch_bounds__(kKtThreads, 1)
+    kmeans_tc_kernel(const __grid_constant__ CUtensorMap tm_q, int BH, int N, int G, int q_block,
+                     const int32_t* __restrict__ off, int C, int iters, float* __restrict__ centroids,
+                     int32_t* __restrict__ counts, uint64_t timeout_ns, int* status) {
+  using namespace isa_dev;
+  using L = KtLayout<CP>;
+  constexpr int D = 128;
+  constexpr int kProducer = 4 * kKtSets;
+  constexpr int NG = CP / 8;  // 8-entry groups per centroid part
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + L::kBar + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  // released[slot]: how many uses of the slot have been handed back
+  volatile uint32_t* released = reinterpret_cast<volatile uint32_t*>(smem + L::kMisc + 16);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t n_items = static_cast<int64_t>(BH) * G;
+
+  if (tid == 0) {
+    for (int i = 0; i < kKtSlots; ++i) released[i] = 0u;
+    for (int i = 0; i < kKtSlots; ++i) {
+      mbar_init(bar(L::kXFull + i), 1);
+      mbar_init(bar(L::kXEmpty + i), 1);
+    }
+    for (int i = 0; i < kKtSets; ++i) mbar_init(bar(L::kMmaDone + i), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // one-hot slots of clusters >= C stay zero, and the counts start at zero
+  for (int i = tid; i < static_cast<int>(kKtSets * L::kOhBytes / 16); i += kKtThreads)
+    reinterpret_cast<uint4*>(smem + L::kOh)[i] = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = tid; i < static_cast<int>(kKtSets * L::kRedBytes / 4); i += kKtThreads)
+    reinterpret_cast<uint32_t*>(smem + L::kRed)[i] = 0u;
+  fence_proxy_async_smem();
+  if (warp == kProducer) {
+    tmem_alloc(smem_addr(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // rows [r0, r0 + n) of group `item`; n = 0 for malformed offsets
+  auto rows_of = [&](int64_t item, int64_t& bh, int& g, int& r0, int& n, bool& malformed) {
+    bh = item / G;
+    g = static_cast<int>(item - bh * G);
+    malformed = false;
+    if (off) {
+      r0 = off[g];
+      const int r1 = off[g + 1];
+      if (r0 < 0 || r1 > N || r1 <= r0) {
+        malformed = true;
+        r0 = 0;
+        n = 0;
+      } else {
+        n = r1 - r0;
+      }
+    } else {
+      r0 = g * q_block;
+      n = min(N, r0 + q_block) - r0;
+    }
+  };
+
+  if (warp == kProducer) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      uint32_t k = 0, loads = 0;
+      for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
+        const uint32_t slot = k % kKtSlots, use = k / kKtSlots;
+        if (!mbar_wait(bar(L::kXEmpty + slot), (use & 1u) ^ 1u, abort_flag, timeout_ns)) break;
+        int64_t bh;
+        int g, r0, n;
+        bool bad;
+        rows_of(item, bh, g, r0, n, bad);
+        if (n >= 1 && n <= 128) {
+          mbar_arrive_expect_tx(bar(L::kXFull + slot), L::kXBytes);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(base + L::kX + slot * L::kXBytes + c * L::kBox, &tm_q, bar(L::kXFull + slot), c * 64, r0,
+                        static_cast<int32_t>(bh));
+        } else {
+          mbar_arrive(bar(L::kXFull + slot));  // nothing to load for this group
+        }
+        loads = k + 1;
+      }
+      if (*abort_flag) {
+        // let the copies already issued land before the CTA leaves
+        const uint32_t first = loads > kKtSlots ? loads - kKtSlots : 0;
+        for (uint32_t i = first; i < loads; ++i) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(bar(L::kXFull + i % kKtSlots), (i / kKtSlots) & 1u))
+            if (global_timer_ns() - t0 > 200000000ull) break;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------- k-means sets
+    const int s = warp >> 2, q4 = warp & 3;
+    const int t = q4 * 32 + lane;  // TMEM lane: the X row (assign) or the dimension (update)
+    // the set's MMA-issuing warp sits on SM sub-partition s, so that no two
+    // issuing warps share one; the next warp finishes the norms and counts
+    const int q_mma = s & 3, q_aux = (s + 1) & 3;
+    const uint32_t bar_id = 1u + static_cast<uint32_t>(s);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint32_t col_s = 64u * s, col_u = 64u * s + 32u;
+    const uint32_t mc = base + L::kMc + s * L::kMcBytes;
+    const uint32_t oh = base + L::kOh + s * L::kOhBytes;
+    uint4* mc_row = reinterpret_cast<uint4*>(smem + L::kMc + s * L::kMcBytes) + t;  // K index t of N group 0
+    uint4* oh_row = reinterpret_cast<uint4*>(smem + L::kOh + s * L::kOhBytes) + t;
+    float* nsq_part = reinterpret_cast<float*>(smem + L::kRed + s * L::kRedBytes);  // [16][4]
+    float* nsq_fin = nsq_part + 64;                                                // [16]
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(nsq_fin + 16);                      // [16]
+    float* inv = reinterpret_cast<float*>(cnt + 16);                               // [16]
+    constexpr uint32_t idesc_assign = idesc_bf16_f32(128, 2 * CP, 1, 0);
+    constexpr uint32_t idesc_update = idesc_bf16_f32(128, 16, 1, 1);
+    uint32_t mma_waits = 0;
+    bool pending = false;  // an MMA batch was committed and not yet waited for
+    bool ok = true;
+    // waits for this set's last MMA batch; the set agrees on the outcome
+    auto wait_mma = [&]() -> bool {
+      bool good = true;
+      if (q4 == q_mma) good = mbar_wait_warp(bar(L::kMmaDone + s), mma_waits & 1u, abort_flag, timeout_ns);
+      good = named_bar_and(bar_id, 128, good);
+      if (good) {
+        ++mma_waits;
+        pending = false;
+        tc_fence_after();
+      }
+      return good;
+    };
+    // The sets take the slots' uses out of order (a set may be through with
+    // a group before the group of the slot's previous use has even landed),
+    // so before waiting on a slot's full barrier for use u a set waits until
+    // uses 0 .. u-1 have been handed back: the barrier is then at most one
+    // phase ahead of u and its parity cannot alias.
+    auto wait_released = [&](uint32_t slot, uint32_t use) -> bool {
+      const uint64_t t0 = global_timer_ns();
+      uint32_t spins = 0;
+      while (released[slot] != use) {
+        if ((++spins & 63u) == 0) {
+          if (*abort_flag) return false;
+          if (global_timer_ns() - t0 > timeout_ns) {
+            *abort_flag = 1;
+            return false;
+          }
+        }
+      }
+      return true;
+    };
+    // hands a slot back to the producer (thread 0 of the set)
+    auto release_slot = [&](uint32_t slot, uint32_t use) {
+      if (t == 0) {
+        released[slot] = use + 1u;
+        __threadfence_block();
+        mbar_arrive(bar(L::kXEmpty + slot));
+      }
+    };
+    uint32_t k = static_cast<uint32_t>(s);
+    for (int64_t item = blockIdx.x + static_cast<int64_t>(s) * gridDim.x; item < n_items && ok;
+         item += static_cast<int64_t>(kKtSets) * gridDim.x, k += kKtSets) {
+      const uint32_t slot = k % kKtSlots, use = k / kKtSlots;
+      int64_t bh;
+      int g, r0, n;
+      bool bad;
+      rows_of(item, bh, g, r0, n, bad);
+      bool got = true;
+      if (q4 == 0) {
+        got = __all_sync(0xffffffffu, wait_released(slot, use));
+        if (got) got = mbar_wait_warp(bar(L::kXFull + slot), use & 1u, abort_flag, timeout_ns);
+      }
+      got = named_bar_and(bar_id, 128, got);
+      if (!got) {
+        ok = false;
+        break;
+      }
+      if (n > 128) {  // a larger group: the warp-per-group kernel runs it
+        release_slot(slot, use);
+        continue;
+      }
+      if (bad && t == 0) atomicCAS(status, 0, kStatusDeviceCheck);
+      const uint32_t xs = base + L::kX + slot * L::kXBytes;
+      const uint8_t* xp = smem + L::kX + slot * L::kXBytes;
+      // thread t's dimension of every centroid, initialised at rows floor(c n / C)
+      float mu[CP];
+#pragma unroll
+      for (int c = 0; c < CP; ++c) {
+        const int r = (c < C && n > 0) ? static_cast<int>((static_cast<int64_t>(c) * n) / C) : -1;
+        mu[c] = r < 0 ? 0.0f : bf16_to_f(*reinterpret_cast<const uint16_t*>(xp + sw128_off(128, r, t)));
+      }
+      uint32_t my_count = 0;  // the count of cluster t (t < C) from the last assignment
+      for (int it = 0; it < iters && n > 0; ++it) {
+        // ---- centroid operands (hi and lo parts, MN-major) and |mu_c|^2 partials
+        {
+          uint32_t hi[CP / 2], lo[CP / 2];
+          float p[CP];
+#pragma unroll
+          for (int j = 0; j < CP / 2; ++j) {
+            hi[j] = pack_bf16x2(mu[2 * j], mu[2 * j + 1]);
+            lo[j] = pack_bf16x2(mu[2 * j] - __uint_as_float(hi[j] << 16),
+                                mu[2 * j + 1] - __uint_as_float(hi[j] & 0xFFFF0000u));
+          }
+#pragma unroll
+          for (int j = 0; j < NG; ++j) {
+            mc_row[j * (L::kNGroup / 16)] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
+            mc_row[(NG + j) * (L::kNGroup / 16)] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
+          }
+#pragma unroll
+          for (int c = 0; c < CP; ++c) p[c] = mu[c] * mu[c];
+          int e;
+          const float ps = warp_sum_scatter<CP>(p, lane, e);
+          if ((lane & (32 / CP - 1)) == 0) nsq_part[e * 4 + q4] = ps;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(bar_id, 128);
+        // ---- S = X [hi | lo]^T, while warp 1 finishes the norms and clears the counts
+        if (q4 == q_mma) {
+          tc_fence_after();
+          const uint64_t da = smem_desc_sw128(xs, 16, 1024), db = smem_desc_none(mc, 128, L::kNGroup);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t oa = ((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4;
+            if (elect_one()) mma_ss(tmem + col_s, da + oa, db + ((kk * 256) >> 4), idesc_assign, kk > 0 ? 1u : 0u);
+          }
+          if (elect_one()) tc_commit(bar(L::kMmaDone + s));
+        } else if (q4 == q_aux && lane < CP) {
+          const float4 np = *reinterpret_cast<const float4*>(nsq_part + 4 * lane);
+          nsq_fin[lane] = (np.x + np.y) + (np.z + np.w);
+          cnt[lane] = 0u;
+        }
+        pending = true;
+        if (!wait_mma()) {
+          ok = false;
+          break;
+        }
+        // ---- assignment: thread t = row t of the tile
+        int label = -1;
+        {
+          uint32_t sv[16];
+          tmem_ld16(lane_base + col_s, sv);
+          uint32_t sv2[16];
+          if constexpr (CP == 16) tmem_ld16(lane_base + col_s + 16, sv2);
+          tmem_wait_ld();
+          float nsq[CP];
+#pragma unroll
+          for (int j = 0; j < CP / 4; ++j) {
+            const float4 v4 = reinterpret_cast<const float4*>(nsq_fin)[j];
+            nsq[4 * j] = v4.x;
+            nsq[4 * j + 1] = v4.y;
+            nsq[4 * j + 2] = v4.z;
+            nsq[4 * j + 3] = v4.w;
+          }
+          float best = INFINITY;
+          int bi = 0;
+#pragma unroll
+          for (int c = 0; c < CP; ++c) {
+            const uint32_t s_hi = CP == 16 ? (c < 16 ? sv[c] : 0u) : sv[c];
+            const uint32_t s_lo = CP == 16 ? sv2[c] : sv[CP + c];
+            const float dot = __uint_as_float(s_hi) + __uint_as_float(s_lo);
+            const float dist = nsq[c] - 2.0f * dot;
+            if (c < C && dist < best) {
+              best = dist;
+              bi = c;
+            }
+          }
+          label = t < n ? bi : -1;
+        }
+        // one-hot row t: slot `label` holds 1.0 (bf16 0x3F80)
+        {
+          const uint32_t w1 = 0x3F80u << ((label & 1) << 4);
+#pragma unroll
+          for (int j = 0; j < NG; ++j) {
+            uint32_t wd[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) wd[i] = (label >> 1) == 4 * j + i ? w1 : 0u;
+            oh_row[j * (L::kNGroup / 16)] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < CP; ++c) {
+          if (c < C) {
+            const uint32_t b = __ballot_sync(0xffffffffu, label == c);
+            if (lane == 0 && b) atomicAdd(&cnt[c], static_cast<uint32_t>(__popc(b)));
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(bar_id, 128);
+        // ---- Sum^T = X^T OH, while warp 1 takes the reciprocal counts
+        if (q4 == q_mma) {
+          tc_fence_after();
+          const uint64_t da = smem_desc_sw128(xs, L::kBox, 1024), db = smem_desc_none(oh, 128, L::kNGroup);
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            if (elect_one())
+              mma_ss(tmem + col_u, da + ((kk * 2048) >> 4), db + ((kk * 256) >> 4), idesc_update, kk > 0 ? 1u : 0u);
+          if (elect_one()) tc_commit(bar(L::kMmaDone + s));
+        } else if (q4 == q_aux && lane < CP) {
+          const uint32_t cc = cnt[lane];
+          inv[lane] = cc > 0u ? 1.0f / static_cast<float>(cc) : 0.0f;
+        }
+        pending = true;
+        if (!wait_mma()) {
+          ok = false;
+          break;
+        }
+        if (it == iters - 1) release_slot(slot, use);  // X is no longer read
+        // ---- update: thread t = dimension t
+        {
+          uint32_t uv[16];
+          tmem_ld16(lane_base + col_u, uv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < CP / 4; ++j) {
+            const float4 i4 = reinterpret_cast<const float4*>(inv)[j];
+            const float iv[4] = {i4.x, i4.y, i4.z, i4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 4 * j + e;
+              if (iv[e] > 0.0f) mu[c] = __uint_as_float(uv[c]) * iv[e];
+            }
+          }
+          if (t < C) my_count = cnt[t];
+        }
+      }
+      if (!ok) break;
+      if (n == 0) release_slot(slot, use);
+      const int64_t o = bh * G + g;
+#pragma unroll
+      for (int c = 0; c < CP; ++c)
+        if (c < C) centroids[(o * C + c) * D + t] = mu[c];
+      if (t < C) counts[o * C + t] = static_cast<int32_t>(my_count);
+    }
+    if (pending && q4 == q_mma) {
+      // a batch whose wait gave up may still be running: let it finish before
+      // the tensor memory is freed
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bar(L::kMmaDone + s), mma_waits & 1u))
+        if (global_timer_ns() - t0 > 200000000ull) break;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort_flag) atomicCAS(status, 0, kStatusTimeout);
+  if (warp == kProducer) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
 
 // ------------------------------------------------------------------ mass
 // One CTA per (batch*head, 128 centroid rows = 128 / Cp groups; Cp = C
@@ -708,6 +1143,43 @@ int launch_mass(const ScoreLaunch& s, int nK, int BH, cudaStream_t stream) {
 }
 
 template <int D>
+int launch_mass_any(const ScoreLaunch& s, int nK, int BH, cudaStream_t stream) {
+  int Cp = 1;
+  while (Cp < s.C) Cp <<= 1;
+  switch (Cp) {
+    case 1: return launch_mass<D, 1>(s, nK, BH, stream);
+    case 2: return launch_mass<D, 2>(s, nK, BH, stream);
+    case 4: return launch_mass<D, 4>(s, nK, BH, stream);
+    case 8: return launch_mass<D, 8>(s, nK, BH, stream);
+    default: return launch_mass<D, 16>(s, nK, BH, stream);
+  }
+}
+
+// The tensor-core k-means over the groups of at most 128 rows (d = 128, C <= 16).
+cudaError_t launch_kmeans_tc(const ScoreLaunch& s, int BH, cudaStream_t stream) {
+  CUtensorMap tq;
+  if (!make_bf16_map(&tq, s.q, BH, s.N, 128, 128)) return cudaErrorInvalidValue;
+  const long long items = static_cast<long long>(BH) * s.G;
+  const int grid = static_cast<int>(items < s.num_sms ? items : s.num_sms);
+  if (s.C <= 8) {
+    using L = KtLayout<8>;
+    const cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kmeans_tc_kernel<8>), L::kAlloc);
+    if (e != cudaSuccess) return e;
+    kmeans_tc_kernel<8><<<grid, kKtThreads, L::kAlloc, stream>>>(tq, BH, s.N, s.G, s.q_block, s.q_offsets, s.C,
+                                                                 s.iters, s.centroids, s.counts, kWaitTimeoutNs,
+                                                                 s.status);
+  } else {
+    using L = KtLayout<16>;
+    const cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kmeans_tc_kernel<16>), L::kAlloc);
+    if (e != cudaSuccess) return e;
+    kmeans_tc_kernel<16><<<grid, kKtThreads, L::kAlloc, stream>>>(tq, BH, s.N, s.G, s.q_block, s.q_offsets, s.C,
+                                                                  s.iters, s.centroids, s.counts, kWaitTimeoutNs,
+                                                                  s.status);
+  }
+  return cudaGetLastError();
+}
+
+template <int D>
 int launch_score_d(const ScoreLaunch& s, cudaStream_t stream) {
   const int BH = s.B * s.H;
   const int nK = (s.N + s.Bk - 1) / s.Bk;
@@ -715,6 +1187,15 @@ int launch_score_d(const ScoreLaunch& s, cudaStream_t stream) {
                                                                             s.Bk, nK, s.kbar_hi, s.kbar_lo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
+  // groups of at most 128 rows (every group of the uniform layouts) take the
+  // tensor-core k-means when d = 128 and C <= 16; the rest, the per-warp one
+  int warp_min_rows = 0;
+  if (D == 128 && s.C <= 16) {
+    e = launch_kmeans_tc(s, BH, stream);
+    if (e != cudaSuccess) return static_cast<int>(e);
+    warp_min_rows = 128;
+    if (!s.q_offsets && s.q_block <= 128) return launch_mass_any<D>(s, nK, BH, stream);
+  }
   using KL = KmLayout<D>;
   int km_blocks_per_sm[2] = {0, 0};
   e = ensure_smem_attr(reinterpret_cast<const void*>(kmeans_warp_kernel<D, 1>), static_cast<int>(KL::kAlloc));
@@ -739,23 +1220,15 @@ int launch_score_d(const ScoreLaunch& s, cudaStream_t stream) {
     if (s.C <= 8)
       kmeans_warp_kernel<D, 1><<<grid, kKmWarps * 32, KL::kAlloc, stream>>>(
           static_cast<const uint16_t*>(s.q), BH, s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids,
-          s.counts, s.status);
+          s.counts, warp_min_rows, s.status);
     else
       kmeans_warp_kernel<D, 2><<<grid, kKmWarps * 32, KL::kAlloc, stream>>>(
           static_cast<const uint16_t*>(s.q), BH, s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids,
-          s.counts, s.status);
+          s.counts, warp_min_rows, s.status);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
-  int Cp = 1;
-  while (Cp < s.C) Cp <<= 1;
-  switch (Cp) {
-    case 1: return launch_mass<D, 1>(s, nK, BH, stream);
-    case 2: return launch_mass<D, 2>(s, nK, BH, stream);
-    case 4: return launch_mass<D, 4>(s, nK, BH, stream);
-    case 8: return launch_mass<D, 8>(s, nK, BH, stream);
-    default: return launch_mass<D, 16>(s, nK, BH, stream);
-  }
+  return launch_mass_any<D>(s, nK, BH, stream);
 }
 
 }  // namespace

@@ -27,6 +27,8 @@
 #include <cstdint>
 
 #include "isa_internal.h"
+#include "mma_sync.cuh"
+#include "ptx.cuh"
 
 namespace isa_impl {
 namespace {
@@ -50,6 +52,26 @@ __device__ __forceinline__ uint64_t philox_word0(uint64_t c0, uint64_t c1, uint6
     k1 += 0xBB67AE8584CAA73BULL;
   }
   return c0;
+}
+
+// w = floor(m / m_max * 2^31) + 1 for a block of the rest with mass bits
+// `key` (0 for non-positive mass), where the quotient is the IEEE fp64
+// division rounded to nearest.  With c31 = RN(2^31 / m_max) the product
+// y = RN(m c31) is within 2^-21 of X = m 2^31 / m_max (X < 2^31, two
+// roundings of at most 2^-53 each), and RN(m / m_max) 2^31 can only reach the
+// next integer above X when X lies within 2^-23 of it.  So when y is more
+// than 2^-20 away from every integer, floor(y) is the rule's value; otherwise
+// (rare) the division itself decides.
+__device__ __noinline__ uint32_t quant_weight_div(uint32_t key, double mmax) {
+  return static_cast<uint32_t>(floor(static_cast<double>(__uint_as_float(key)) / mmax * 2147483648.0)) + 1u;
+}
+__device__ __forceinline__ uint32_t quant_weight(uint32_t key, double mmax, double c31) {
+  if (!(mmax > 0.0) || key == 0u) return 1u;
+  const double y = static_cast<double>(__uint_as_float(key)) * c31;
+  const double fl = floor(y);
+  const double fr = y - fl;  // exact: fl <= y < fl + 1
+  if (fr > 0x1p-20 && fr < 1.0 - 0x1p-20) return static_cast<uint32_t>(fl) + 1u;
+  return quant_weight_div(key, mmax);
 }
 
 struct SelShared {
@@ -221,14 +243,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
       if (!(flag[i] & 1)) kmax = max(kmax, key[i]);
     kmax = block_max_u32(kmax, sh);
     const double mmax = static_cast<double>(__uint_as_float(kmax));
-    for (int i = i0; i < i1; ++i) {
-      uint32_t w = 0;
-      if (!(flag[i] & 1))
-        w = mmax > 0.0 ? static_cast<uint32_t>(floor(static_cast<double>(__uint_as_float(key[i])) / mmax *
-                                                     2147483648.0)) + 1u
-                       : 1u;
-      wq[i] = w;
-    }
+    const double c31 = mmax > 0.0 ? 2147483648.0 / mmax : 0.0;
+    for (int i = i0; i < i1; ++i) wq[i] = (flag[i] & 1) ? 0u : quant_weight(key[i], mmax, c31);
     int n_capped = 0;
     for (;;) {
       uint64_t t = 0;
@@ -283,10 +299,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
     }
   }
 
-  // ---- write the plan row: exact ascending, then capped + drawn ascending
+  // ---- write the plan row: exact ascending, then capped + drawn ascending.
+  // The drawn blocks' log-weights are left to a second, converged pass over
+  // the rest part of the row: per rest position, the drawn block's weight (0
+  // for a capped block) goes to a list over the key array, which nothing
+  // reads any more.
   int32_t* out_idx = a.idx + row * S;
   float* out_lw = a.log_w + row * S;
-  const double lnT = T > 0 ? log(static_cast<double>(T)) : 0.0;
+  const int n_rs = S - n_exact;
   uint64_t ne = 0, nr = 0;
   for (int i = i0; i < i1; ++i) {
     const uint8_t f = flag[i];
@@ -294,8 +314,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
     nr += (!(f & 1) && (f & 6)) ? 1u : 0u;
   }
   uint64_t tot;
-  const uint64_t pre = block_scan_u64((ne << 32) | nr, sh, &tot);  // both counts < 2^32
-  uint64_t pe = pre >> 32, pr = static_cast<uint64_t>(n_exact) + (pre & 0xFFFFFFFFull);
+  const uint64_t pre = block_scan_u64((ne << 32) | nr, sh, &tot);  // both counts < 2^32 (its barriers also
+                                                                  // order every key read before the list)
+  uint64_t pe = pre >> 32, pr = pre & 0xFFFFFFFFull;
+  uint32_t* wl = key;
   for (int i = i0; i < i1; ++i) {
     const uint8_t f = flag[i];
     if (f & 1) {
@@ -305,15 +327,22 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
       }
       ++pe;
     } else if (f & 6) {
-      if (pr < static_cast<uint64_t>(S)) {
-        out_idx[pr] = i;
-        out_lw[pr] = (f & 4) ? static_cast<float>(lnT - log(static_cast<double>(static_cast<uint64_t>(n_left) * wq[i])))
-                             : 0.0f;
+      if (pr < static_cast<uint64_t>(n_rs)) {
+        out_idx[n_exact + pr] = i;
+        wl[pr] = (f & 4) ? wq[i] : 0u;
       }
       ++pr;
     }
   }
+  __syncthreads();
   const uint64_t tot_e = tot >> 32, tot_r = tot & 0xFFFFFFFFull;
+  const double lnT = T > 0 ? log(static_cast<double>(T)) : 0.0;
+  const int n_w = static_cast<int>(tot_r < static_cast<uint64_t>(n_rs) ? tot_r : static_cast<uint64_t>(n_rs));
+  for (int k = tid; k < n_w; k += kSelThreads) {
+    const uint32_t wv = wl[k];
+    out_lw[n_exact + k] =
+        wv ? static_cast<float>(lnT - log(static_cast<double>(static_cast<uint64_t>(n_left) * wv))) : 0.0f;
+  }
   if (tid == 0) {
     if (sh.bad || tot_e != static_cast<uint64_t>(n_exact) || tot_e + tot_r != static_cast<uint64_t>(S))
       atomicCAS(a.status, 0, kStatusDeviceCheck);
@@ -355,22 +384,15 @@ __device__ __forceinline__ uint32_t warp_excl_u32(uint32_t v, int lane) {
   return inc - v;
 }
 
+// One plan row by one warp.  st: the row's mass as staged by the caller
+// (element i at i + i / 32, so that the lanes' blocked reads are free of bank
+// conflicts), reused for the log-weight list once the keys are in registers;
+// hist: the warp's 256-bin radix histogram.
 template <int VPL>
-__global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(SelectLaunch a) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarpRowsPerCta + warp;
-  const int64_t rows = static_cast<int64_t>(a.B) * a.H * a.G;
-  if (row >= rows) return;
+__device__ __forceinline__ void select_row_warp(const SelectLaunch& a, const int64_t row, uint32_t* st,
+                                                uint32_t* hist, const int lane) {
   const int nK = a.nK;
-  // this warp's shared slice, skewed by one word per 32 so that the blocked
-  // per-lane reads are free of bank conflicts: first the mass row, then the
-  // integer weights of the rest
-  uint32_t* st = reinterpret_cast<uint32_t*>(sm) + warp * (32 * VPL + VPL);
   auto at = [](int i) { return i + (i >> 5); };
-  const float* m = a.mass + row * nK;
-  for (int i = lane; i < nK; i += 32) st[at(i)] = __float_as_uint(m[i]);
-  __syncwarp();
   const int g = static_cast<int>(row % a.G);
   const int h = static_cast<int>((row / a.G) % a.H);
   const int b = static_cast<int>(row / (static_cast<int64_t>(a.G) * a.H));
@@ -402,7 +424,6 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
     // from the top: a 256-bin histogram of the keys that match the prefix
     // so far, and the bin holding the remaining rank (lane l owns bins
     // 8l .. 8l+7, so the bins above a lane's are those of higher lanes)
-    uint32_t* hist = reinterpret_cast<uint32_t*>(sm) + kWarpRowsPerCta * (32 * VPL + VPL) + warp * 256;
     uint32_t t = 0, mask = 0, kk = static_cast<uint32_t>(n_exact);
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
@@ -464,14 +485,17 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
       }
     }
   }
-  // ---- the rest: weights (into the shared slice), capping, systematic PPS
+  // ---- the rest: weights (in registers, in place of the keys), capping,
+  // systematic PPS.  Every loop over the lane's blocks is unrolled, so the
+  // per-block flags are bits at constant positions.
   const int n_rest = nK - n_exact;
   uint64_t cap = 0, drawn = 0;  // bit v: capped (or taken whole), drawn
   uint64_t T = 0;
   int n_left = 0;
   if (n_sample >= n_rest) {
-    for (int v = 0; v < nv; ++v)
-      if (!((ex >> v) & 1)) cap |= 1ull << v;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
+      if (v < nv && !((ex >> v) & 1)) cap |= 1ull << v;
   } else if (n_sample > 0) {
     uint32_t kmax = 0;
 #pragma unroll
@@ -479,30 +503,28 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
       if (v < nv && !((ex >> v) & 1)) kmax = max(kmax, key[v]);
     kmax = __reduce_max_sync(0xffffffffu, kmax);
     const double mmax = static_cast<double>(__uint_as_float(kmax));
-    __syncwarp();
+    const double c31 = mmax > 0.0 ? 2147483648.0 / mmax : 0.0;
+    // w = floor(m / m_max * 2^31) + 1 on the rest; 0 on the exact set and past the row
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
-      if (v < nv) {
-        uint32_t wv = 0;
-        if (!((ex >> v) & 1))
-          wv = mmax > 0.0 ? static_cast<uint32_t>(floor(static_cast<double>(__uint_as_float(key[v])) / mmax *
-                                                       2147483648.0)) + 1u
-                          : 1u;
-        st[at(base + v)] = wv;  // 0 marks exact blocks
-      }
+      uint32_t wv = 0;
+      if (v < nv && !((ex >> v) & 1)) wv = quant_weight(key[v], mmax, c31);
+      key[v] = wv;
     }
     int n_capped = 0;
+    uint64_t tl = 0;  // after the loop: this lane's total over the uncapped rest
     for (;;) {
-      uint64_t tl = 0;
-      for (int v = 0; v < nv; ++v)
-        if (!((cap >> v) & 1)) tl += st[at(base + v)];
+      tl = 0;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v)
+        if (!((cap >> v) & 1)) tl += key[v];
       T = warp_sum_u64(tl);
       n_left = n_sample - n_capped;
       uint32_t add = 0;
       uint64_t newcap = 0;
-      for (int v = 0; v < nv; ++v) {
-        const uint32_t wv = st[at(base + v)];
-        if (wv != 0 && !((cap >> v) & 1) && static_cast<uint64_t>(n_left) * wv >= T) {
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        if (key[v] != 0 && !((cap >> v) & 1) && static_cast<uint64_t>(n_left) * key[v] >= T) {
           newcap |= 1ull << v;
           ++add;
         }
@@ -518,45 +540,45 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
                        a.seed, 0) >>
           32);
       const uint64_t nl = static_cast<uint64_t>(n_left);
-      const uint64_t ut_lo = static_cast<uint64_t>(U) * T;  // U T < 2^76
-      const uint64_t ut_hi = __umul64hi(static_cast<uint64_t>(U), T);
       // points of the comb below x: q + [r 2^32 > U T] with q = floor(x n' / T)
-      // and r = x n' - q T.  Walking x up by an uncapped weight (n' w < T)
-      // moves r up by n' w and needs at most one reduction by T, so only the
-      // start of each lane's segment takes a division.
-      auto above = [&](uint64_t r_) -> bool {
-        const uint64_t r_hi = r_ >> 32, r_lo = r_ << 32;
-        return r_hi > ut_hi || (r_hi == ut_hi && r_lo > ut_lo);
-      };
-      uint64_t local = 0;
-      for (int v = 0; v < nv; ++v)
-        if (!((cap >> v) & 1)) local += st[at(base + v)];
-      const uint64_t xn0 = warp_excl_u64(local, lane) * nl;
-      uint64_t q = xn0 / T, r = xn0 - q * T;
-      uint64_t f_prev = q + (above(r) ? 1u : 0u);
-      for (int v = 0; v < nv; ++v) {
-        const uint32_t wv = st[at(base + v)];
-        if (wv != 0 && !((cap >> v) & 1)) {
-          r += static_cast<uint64_t>(wv) * nl;
+      // and r = x n' - q T; r 2^32 > U T is r > floor(U T / 2^32) for whole r.
+      // Walking x up by an uncapped weight (n' w < T) moves r up by n' w and
+      // needs at most one reduction by T, so only the start of each lane's
+      // segment takes a division.
+      const uint64_t thr = static_cast<uint64_t>(U) * (T >> 32) + ((static_cast<uint64_t>(U) * (T & 0xFFFFFFFFull)) >> 32);
+      const uint64_t xn0 = warp_excl_u64(tl, lane) * nl;
+      uint64_t r = xn0 % T;
+      uint32_t q = static_cast<uint32_t>(xn0 / T);  // at most n'
+      uint32_t f_prev = q + (r > thr ? 1u : 0u);
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        if (key[v] != 0 && !((cap >> v) & 1)) {
+          r += static_cast<uint64_t>(key[v]) * nl;
           if (r >= T) {
             r -= T;
             ++q;
           }
-          const uint64_t f = q + (above(r) ? 1u : 0u);
+          const uint32_t f = q + (r > thr ? 1u : 0u);
           if (f != f_prev) drawn |= 1ull << v;
           f_prev = f;
         }
       }
     }
   }
-  // ---- write the plan row: exact ascending, then capped + drawn ascending
+  // ---- write the plan row: exact ascending, then capped + drawn ascending.
+  // The drawn blocks' log-weights are left to a second, converged pass over
+  // the rest part of the row: each lane records, per rest position it fills,
+  // the drawn block's weight (0 for a capped block) in the warp's shared
+  // slice, which no longer holds anything the warp reads.
   int32_t* out_idx = a.idx + row * S;
   float* out_lw = a.log_w + row * S;
+  const int n_rs = S - n_exact;
   const uint32_t ne = __popcll(ex), nr = __popcll(cap | drawn);
   uint32_t pe = warp_excl_u32(ne, lane);
-  uint32_t pr = static_cast<uint32_t>(n_exact) + warp_excl_u32(nr, lane);
-  const double lnT = T > 0 ? log(static_cast<double>(T)) : 0.0;
-  for (int v = 0; v < nv; ++v) {
+  uint32_t pr = warp_excl_u32(nr, lane);
+  __syncwarp();
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
     const int i = base + v;
     if ((ex >> v) & 1) {
       if (pe < static_cast<uint32_t>(n_exact)) {
@@ -565,19 +587,63 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) select_warp_kernel(Selec
       }
       ++pe;
     } else if (((cap | drawn) >> v) & 1) {
-      if (pr < static_cast<uint32_t>(S)) {
-        out_idx[pr] = i;
-        out_lw[pr] = ((drawn >> v) & 1) ? static_cast<float>(lnT - log(static_cast<double>(
-                                                                        static_cast<uint64_t>(n_left) * st[at(i)])))
-                                        : 0.0f;
+      if (pr < static_cast<uint32_t>(n_rs)) {
+        out_idx[n_exact + pr] = i;
+        st[pr] = ((drawn >> v) & 1) ? key[v] : 0u;
       }
       ++pr;
     }
   }
+  __syncwarp();
   const uint32_t tot_e = __reduce_add_sync(0xffffffffu, ne), tot_r = __reduce_add_sync(0xffffffffu, nr);
+  const double lnT = T > 0 ? log(static_cast<double>(T)) : 0.0;
+  const int n_w = min(static_cast<int>(tot_r), n_rs);
+  for (int k = lane; k < n_w; k += 32) {
+    const uint32_t wv = st[k];
+    out_lw[n_exact + k] =
+        wv ? static_cast<float>(lnT - log(static_cast<double>(static_cast<uint64_t>(n_left) * wv))) : 0.0f;
+  }
   const bool any_bad = __any_sync(0xffffffffu, bad);
   if (lane == 0 && (any_bad || tot_e != static_cast<uint32_t>(n_exact) || tot_e + tot_r != static_cast<uint32_t>(S)))
     atomicCAS(a.status, 0, kStatusDeviceCheck);
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// Persistent warps: warp w of the grid takes rows w, w + W, w + 2W, ... (W =
+// the grid's warps) and stages the next row's mass in its second shared
+// buffer (cp.async) while it selects the current one.
+template <int VPL>
+__global__ void __launch_bounds__(32 * kWarpRowsPerCta, VPL <= 40 ? 2 : 1) select_warp_kernel(SelectLaunch a) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  constexpr int kSlice = 32 * VPL + VPL;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(a.B) * a.H * a.G;
+  uint32_t* st = reinterpret_cast<uint32_t*>(sm) + warp * 2 * kSlice;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sm) + kWarpRowsPerCta * 2 * kSlice + warp * 256;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarpRowsPerCta;
+  int64_t row = static_cast<int64_t>(blockIdx.x) * kWarpRowsPerCta + warp;
+  auto stage = [&](int64_t r, uint32_t* dst) {
+    const float* m = a.mass + r * a.nK;
+    for (int i = lane; i < a.nK; i += 32) cp_async4(isa_dev::smem_addr(dst + i + (i >> 5)), m + i);
+  };
+  using isa_dev::cp_async_commit;
+  using isa_dev::cp_async_wait_group;
+  if (row < rows) stage(row, st);
+  cp_async_commit();
+  int buf = 0;
+  for (; row < rows; row += stride) {
+    if (row + stride < rows) stage(row + stride, st + (buf ^ 1) * kSlice);
+    cp_async_commit();
+    cp_async_wait_group<1>();  // this lane's copies of the current row have landed
+    __syncwarp();
+    select_row_warp<VPL>(a, row, st + buf * kSlice, hist, lane);
+    __syncwarp();  // the buffer is restaged only after every lane is done with it
+    buf ^= 1;
+  }
+  cp_async_wait_group<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -665,12 +731,19 @@ __global__ void __launch_bounds__(kSelThreads) top_p_count_kernel(const float* _
 template <int VPL>
 int launch_select_warp(const SelectLaunch& s, cudaStream_t stream) {
   const long long rows = static_cast<long long>(s.B) * s.H * s.G;
-  const size_t smem = static_cast<size_t>(kWarpRowsPerCta) * (32 * VPL + VPL + 256) * 4;
+  const size_t smem = static_cast<size_t>(kWarpRowsPerCta) * (2 * (32 * VPL + VPL) + 256) * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_warp_kernel<VPL>), static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
   }
-  const unsigned grid = static_cast<unsigned>((rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta);
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_warp_kernel<VPL>,
+                                                                32 * kWarpRowsPerCta, smem);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  if (per_sm < 1) return static_cast<int>(cudaErrorInvalidConfiguration);
+  const long long want = (rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta;
+  const long long cap = static_cast<long long>(s.num_sms > 0 ? s.num_sms : 148) * per_sm;
+  const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
   select_warp_kernel<VPL><<<grid, 32 * kWarpRowsPerCta, smem, stream>>>(s);
   return static_cast<int>(cudaGetLastError());
 }
