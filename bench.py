@@ -472,6 +472,27 @@ def main():
     for v_ in stages.values():
         v_["frac_hbm"] = v_["gbs"] / hbm
 
+    # score -> select in one call (isa_plan): the mass stays in L2, in chunks
+    # of heads, and never reaches HBM
+    if rank == 0:
+        pp = isa.params(w.n_clusters, w.n_iters, w.n_exact, w.n_sample, w.seed)
+        pn = isa.plan_workspace_bytes(lay, pp)
+        pws = torch.empty(pn + 256, dtype=torch.uint8, device=dev)
+        isa.plan(q, k, lay, pp, idx=idx, log_w=lw, workspace=pws, ctx=ctx)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            isa.plan(q, k, lay, pp, idx=idx, log_w=lw, workspace=pws, ctx=ctx)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        st = ctx.sync_status()
+        if st != isa.ISA_OK:
+            raise RuntimeError("device status after isa_plan: %s" % isa.status_string(st))
+        stages["plan"] = {"ms": e0.elapsed_time(e1) / 3, "score_plus_select_ms": score_ms + select_ms,
+                          "workspace_bytes": pn, "mass_bytes_not_allocated": 4 * B * H * G * nK,
+                          "what": "isa_plan: score and select in chunks of heads, mass kept in L2"}
+        del pws
+
     # plan reuse across calls: score + select once, then r attention calls
     # with that plan on activations that change from call to call (two input
     # sets, the second a perturbed copy of the first, taken in turn), timed as

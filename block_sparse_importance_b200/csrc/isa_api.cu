@@ -208,7 +208,7 @@ isa_status do_score(isa_context* ctx, const isa_shape* s, const void* q, const v
 
 isa_status do_select(isa_context* ctx, const isa_shape* s, const float* mass, int32_t ne, int32_t ns, uint64_t seed,
                      int32_t* idx, float* log_w, cudaStream_t st, int h_base = 0, int b_base = 0,
-                     const int32_t* ne_rows = nullptr) {
+                     const int32_t* ne_rows = nullptr, bool discard_mass = false) {
   ISA_TRY(check_ptr(ctx, mass, "mass", 4));
   ISA_TRY(check_ptr(ctx, idx, "idx", 4));
   ISA_TRY(check_ptr(ctx, log_w, "log_w", 4));
@@ -232,6 +232,7 @@ isa_status do_select(isa_context* ctx, const isa_shape* s, const float* mass, in
   l.ne_rows = ne_rows;
   l.status = ctx->d_status;
   l.num_sms = ctx->num_sms;
+  l.discard_mass = discard_mass ? 1 : 0;
   return cuda_status(ctx, launch_select(l, st), "isa_select");
 }
 
@@ -318,6 +319,24 @@ isa_status do_pipeline(isa_context* ctx, const isa_shape* s, const isa_params* p
   ISA_TRY(do_score(ctx, s, q, k, p->n_clusters, p->n_iters, mass, nullptr, nullptr, sws, score_ws, st));
   ISA_TRY(do_select(ctx, s, mass, p->n_exact, p->n_sample, p->seed, idx, lw, st, h_base, b_base));
   return do_attention(ctx, s, q, k, v, idx, lw, static_cast<int32_t>(S), out, lse, aws, attn_ws_bytes(s), false, st);
+}
+
+// isa_plan: heads per chunk, so that one chunk's mass stays well inside L2
+// between the mass kernel that writes it and the selector that reads it.
+constexpr size_t kPlanChunkMassBytes = size_t(48) << 20;
+
+int plan_chunk_heads(const isa_shape* s) {
+  const size_t per_head = static_cast<size_t>(s->num_groups) * nblocks(s) * 4;
+  size_t hc = per_head ? kPlanChunkMassBytes / per_head : 1;
+  if (hc < 1) hc = 1;
+  if (hc > static_cast<size_t>(s->heads)) hc = static_cast<size_t>(s->heads);
+  return static_cast<int>(hc);
+}
+
+size_t plan_bytes(const isa_shape* s, const isa_params* p) {
+  const int hc = plan_chunk_heads(s);
+  return round_up(score_workspace_bytes(1, hc, s->seq_len, s->head_dim, s->num_groups, s->k_block, p->n_clusters)) +
+         round_up(static_cast<size_t>(hc) * s->num_groups * nblocks(s) * 4);
 }
 
 }  // namespace
@@ -598,6 +617,57 @@ isa_status isa_dense_attention(isa_context* ctx, const isa_shape* shape, const v
   if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
   return do_attention(ctx, shape, q, k, v, nullptr, nullptr, 0, out, lse, nullptr, 0, true,
                       static_cast<cudaStream_t>(stream));
+}
+
+size_t isa_plan_workspace_bytes(const isa_shape* s, const isa_params* p) {
+  if (!s || !p || p->n_clusters < 1 || s->heads < 1 || s->num_groups < 1 || s->k_block < 1) return 0;
+  return plan_bytes(s, p);
+}
+
+isa_status isa_plan(isa_context* ctx, const isa_shape* shape, const isa_params* params, const void* q, const void* k,
+                    int32_t* idx, float* log_w, void* workspace, size_t workspace_bytes, void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  if (!params) return fail(ctx, ISA_ERR_INVALID_ARG, "params is NULL");
+  if (params->n_clusters < 1 || params->n_clusters > 16) return fail(ctx, ISA_ERR_INVALID_ARG, "n_clusters must be 1..16");
+  ISA_TRY(check_ptr(ctx, q, "q", 16));
+  ISA_TRY(check_ptr(ctx, k, "k", 16));
+  ISA_TRY(check_ptr(ctx, idx, "idx", 4));
+  ISA_TRY(check_ptr(ctx, log_w, "log_w", 4));
+  const size_t need = plan_bytes(shape, params);
+  if (!workspace || workspace_bytes < need)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "plan workspace %zu bytes < %zu needed", workspace_bytes, need);
+  if (!aligned(workspace, 256)) return fail(ctx, ISA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = shape->heads, hc = plan_chunk_heads(shape);
+  const size_t G = static_cast<size_t>(shape->num_groups), S = static_cast<size_t>(params->n_exact) + params->n_sample;
+  const size_t head_elems = static_cast<size_t>(shape->seq_len) * shape->head_dim;
+  const size_t score_ws = round_up(
+      score_workspace_bytes(1, hc, shape->seq_len, shape->head_dim, shape->num_groups, shape->k_block, params->n_clusters));
+  char* w = static_cast<char*>(workspace);
+  float* mass = reinterpret_cast<float*>(w + score_ws);
+  // Chunks of heads: score the chunk into the chunk-sized mass buffer, then
+  // select from it while it is still in L2; the selector drops every line it
+  // has read, so the mass is not written back to HBM.  Heads are independent
+  // and the uniforms are keyed by the global head and batch index, so the
+  // plan is the one isa_select(isa_score(.)) gives on the whole layer.
+  for (int b = 0; b < shape->batch; ++b) {
+    for (int h0 = 0; h0 < H; h0 += hc) {
+      const int nh = H - h0 < hc ? H - h0 : hc;
+      isa_shape sub = *shape;
+      sub.batch = 1;
+      sub.heads = nh;
+      const size_t bh0 = static_cast<size_t>(b) * H + h0;
+      const char* qc = static_cast<const char*>(q) + bh0 * head_elems * 2;
+      const char* kc = static_cast<const char*>(k) + bh0 * head_elems * 2;
+      ISA_TRY(do_score(ctx, &sub, qc, kc, params->n_clusters, params->n_iters, mass, nullptr, nullptr, w, score_ws,
+                       st));
+      ISA_TRY(do_select(ctx, &sub, mass, params->n_exact, params->n_sample, params->seed, idx + bh0 * G * S,
+                        log_w + bh0 * G * S, st, h0, b, nullptr, true));
+    }
+  }
+  return ISA_OK;
 }
 
 size_t isa_pipeline_workspace_bytes(const isa_shape* s, const isa_params* p) {

@@ -63,6 +63,9 @@ struct SelectLaunch {
   const int32_t* ne_rows;
   int* status;
   int num_sms;
+  // the mass is scratch: once a row has been read, its whole 128-byte lines
+  // are dropped from L2 without being written back (discard.global.L2)
+  int discard_mass;
 };
 int launch_select(const SelectLaunch& s, cudaStream_t stream);
 // Exact-set sizes under the top-p rule, one per plan row, into ne_rows.

@@ -74,6 +74,15 @@ __device__ __forceinline__ uint32_t quant_weight(uint32_t key, double mmax, doub
   return quant_weight_div(key, mmax);
 }
 
+// Drops from L2, without write-back, every whole 128-byte line of a mass row
+// that has been read in full (lines shared with a neighbouring row stay).
+__device__ __forceinline__ void discard_row_lines(const float* row, int nK, int t, int nt) {
+  const uintptr_t s0 = reinterpret_cast<uintptr_t>(row), s1 = s0 + static_cast<uintptr_t>(nK) * 4;
+  const uintptr_t l0 = (s0 + 127) & ~static_cast<uintptr_t>(127), l1 = s1 & ~static_cast<uintptr_t>(127);
+  for (uintptr_t p = l0 + static_cast<uintptr_t>(t) * 128; p < l1; p += static_cast<uintptr_t>(nt) * 128)
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 struct SelShared {
   uint64_t red64[kSelWarps];
   uint32_t red32[kSelWarps];
@@ -170,6 +179,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
     flag[i] = 0;
   }
   __syncthreads();
+  if (a.discard_mass) discard_row_lines(m, nK, tid, kSelThreads);
 
   // ---- exact set: the n_exact largest keys, ties to the lower index
   if (n_exact > 0) {
@@ -639,6 +649,7 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, VPL <= 40 ? 2 : 1) selec
     cp_async_commit();
     cp_async_wait_group<1>();  // this lane's copies of the current row have landed
     __syncwarp();
+    if (a.discard_mass) discard_row_lines(a.mass + row * a.nK, a.nK, lane, 32);
     select_row_warp<VPL>(a, row, st + buf * kSlice, hist, lane);
     __syncwarp();  // the buffer is restaged only after every lane is done with it
     buf ^= 1;

@@ -59,7 +59,12 @@ def clustered_values(w, B: int, H: int, N: int, d: int, device: str = "cuda") ->
 
 
 def run(workload: str = "wan13", heads: int = 4, temps=(0.5, 1.0, 2.0, 4.0, 8.0), seeds=(0, 1, 2, 3),
-        density: float = 0.1, values: str = "clustered") -> dict:
+        density: float = 0.1, values: str = "clustered", keep_plans: bool = False) -> dict:
+    """The study's table.  With keep_plans, every row also carries the plans
+    it measured (CPU tensors: "plans" maps a plan name to a list of (idx,
+    log_w, k_block), one per seed where the row averages over seeds) and the
+    result carries the q, k, v it used, so that the figures can be recomputed
+    elsewhere."""
     w = wl.preset(workload)
     inp = wl.make_inputs(w, "cuda", heads=heads)
     q, k, v = inp.q, inp.k, inp.v
@@ -77,16 +82,25 @@ def run(workload: str = "wan13", heads: int = 4, temps=(0.5, 1.0, 2.0, 4.0, 8.0)
         ns = total - ne
         mass = isa.score(q, k, lay, w.n_clusters, w.n_iters)
         row = {"t": t, "S": total, "n_exact": ne, "n_sample": ns}
+        plans = {"is": [], "unweighted": [], "top_s": [], "is_small_blk": []}
+
+        def keep(name, idx_, lw_, bk):
+            if keep_plans:
+                plans[name].append((idx_.cpu(), lw_.cpu(), bk))
+
         errs = []
         for s in seeds:
             idx, lw = isa.select(mass, lay, ne, ns, s)
             errs.append(rel_l2(isa.attention(q, k, v, idx, lw, lay), dense))
+            keep("is", idx, lw, w.k_block)
             if s == seeds[0]:
                 row["unweighted"] = rel_l2(isa.attention(q, k, v, idx, torch.zeros_like(lw), lay), dense)
+                keep("unweighted", idx, torch.zeros_like(lw), w.k_block)
         row["is"] = sum(errs) / len(errs)
         row["is_seed_spread"] = max(errs) - min(errs)
         idx, lw = isa.select(mass, lay, total, 0, 0)
         row["top_s"] = rel_l2(isa.attention(q, k, v, idx, lw, lay), dense)
+        keep("top_s", idx, lw, w.k_block)
         # four times as many blocks a quarter as tall (the same key rows)
         bk4 = w.k_block // 4
         lay4 = isa.layout_for(q, bk4, w.q_block, scale=scale)
@@ -98,12 +112,19 @@ def run(workload: str = "wan13", heads: int = 4, temps=(0.5, 1.0, 2.0, 4.0, 8.0)
         for s in seeds:
             idx4, lw4 = isa.select(mass4, lay4, ne4, total4 - ne4, s)
             errs4.append(rel_l2(isa.attention(q, k, v, idx4, lw4, lay4), dense))
+            keep("is_small_blk", idx4, lw4, bk4)
         row["is_small_blk"] = sum(errs4) / len(errs4)
         row["small_blk_S"] = total4
+        if keep_plans:
+            row["plans"] = plans
         rows.append(row)
     status = isa.context().sync_status()
-    return {"workload": workload, "heads": heads, "N": N, "k_block": w.k_block, "density": density,
-            "values": values, "seeds": list(seeds), "rows": rows, "status": status}
+    res = {"workload": workload, "heads": heads, "N": N, "k_block": w.k_block, "density": density,
+           "values": values, "seeds": list(seeds), "rows": rows, "status": status}
+    if keep_plans:
+        res["qkv"] = tuple(x.cpu() for x in (q, k, v))
+        res["offsets"] = inp.offsets
+    return res
 
 
 def main():

@@ -79,6 +79,9 @@ def lib():
             L.isa_attention_workspace_bytes.restype = _sz
             L.isa_attention.argtypes = [_P, S, _P, _P, _P, _P, _P, _i32, _P, _P, _P, _sz, _P]
             L.isa_dense_attention.argtypes = [_P, S, _P, _P, _P, _P, _P, _P]
+            L.isa_plan_workspace_bytes.argtypes = [S, Pp]
+            L.isa_plan_workspace_bytes.restype = _sz
+            L.isa_plan.argtypes = [_P, S, Pp, _P, _P, _P, _P, _P, _sz, _P]
             L.isa_pipeline_workspace_bytes.argtypes = [S, Pp]
             L.isa_pipeline_workspace_bytes.restype = _sz
             L.isa_pipeline.argtypes = [_P, S, Pp, _P, _P, _P, _P, _P, _P, _P, _P, _sz, _P]
@@ -409,6 +412,30 @@ def pipeline_workspace_bytes(lay: Layout, p: Params) -> int:
 
 def pipeline_host_workspace_bytes(lay: Layout, p: Params) -> int:
     return int(lib().isa_pipeline_host_workspace_bytes(ctypes.byref(lay.c()), ctypes.byref(p)))
+
+
+def plan_workspace_bytes(lay: Layout, p: Params) -> int:
+    sh = lay.c()
+    return int(lib().isa_plan_workspace_bytes(ctypes.byref(sh), ctypes.byref(p)))
+
+
+def plan(q, k, lay: Layout, p: Params, idx=None, log_w=None, workspace=None, ctx: Optional[Context] = None,
+         stream=None):
+    """isa_plan: score -> select in one call; returns (idx, log_w) [B,H,G,S]."""
+    ctx = ctx or context(q.device.index or 0)
+    for t, n in ((q, "q"), (k, "k")):
+        _dev(t, torch.bfloat16, n)
+    S = p.n_exact + p.n_sample
+    shp = (lay.batch, lay.heads, lay.num_groups, S)
+    idx = idx if idx is not None else _empty(shp, torch.int32, q.device)
+    log_w = log_w if log_w is not None else _empty(shp, torch.float32, q.device)
+    nb = plan_workspace_bytes(lay, p)
+    workspace = _workspace(nb, q.device, workspace)
+    sh = lay.c()
+    st = lib().isa_plan(ctx.handle, ctypes.byref(sh), ctypes.byref(p), _ptr(q), _ptr(k), _ptr(idx), _ptr(log_w),
+                        _ptr(workspace), nb, _stream(stream))
+    ctx.check(st, "isa_plan")
+    return idx, log_w
 
 
 def pipeline(q, k, v, lay: Layout, p: Params, out=None, lse=None, plan_idx=None, plan_log_w=None,

@@ -290,6 +290,24 @@ ISA_API isa_status isa_dense_attention(isa_context* ctx, const isa_shape* shape,
                                const void* k, const void* v, void* out, float* lse, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * isa_plan -- score -> select in one call: the plan of every query group
+ * straight from q and k ("AB-Attention": the selector's estimates feed the
+ * sampler directly; plans are made from the current activations and may then
+ * serve several attention calls).  The result equals isa_select(isa_score(.))
+ * bit for bit, but the estimated mass never reaches HBM: the layer is
+ * scored and selected in chunks of heads whose mass (at most 48 MiB, at
+ * least one head) stays in L2 between the two steps, and the selector drops
+ * every mass line it has read from L2 without writing it back.  The
+ * workspace (isa_plan_workspace_bytes, 256-byte aligned) holds one chunk's
+ * scorer scratch and mass, so it is also much smaller than the whole mass
+ * tensor.  idx, log_w: [B,H,G,S] as isa_select writes them.
+ * ------------------------------------------------------------------------- */
+ISA_API size_t isa_plan_workspace_bytes(const isa_shape* shape, const isa_params* params);
+ISA_API isa_status isa_plan(isa_context* ctx, const isa_shape* shape, const isa_params* params,
+                    const void* q, const void* k, int32_t* idx, float* log_w, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * isa_pipeline -- score -> select -> attention in one call on device
  * buffers (the whole hot path of one attention layer).  The mass tensor,
  * the plan and the scorer's scratch are carved from `workspace`
