@@ -606,7 +606,12 @@ def main():
         inp_cpu = wl.make_inputs(w, "cpu", heads=1)
         cpu = cpu_oracle_sample(w, inp_cpu, target_s=args.ref_seconds)
 
-    launches_per_step = 5 + (1 if aws_n else 0)
+    # key means, k-means (tensor-core kernel for groups of at most 128 rows at
+    # d = 128, C <= 16; the per-warp kernel for the rest), mass, selector,
+    # attention (+ its tile list for clusters or groups above 128 rows)
+    tc_km = d == 128 and w.n_clusters <= 16
+    warp_km = (not tc_km) or w.variable_groups or w.q_block > 128
+    launches_per_step = 4 + int(tc_km) + int(warp_km) + (1 if aws_n else 0)
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",

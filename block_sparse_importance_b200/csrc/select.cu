@@ -369,52 +369,81 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
 // select_kernel.
 constexpr int kWarpRowsPerCta = 8;
 
-__device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-// exclusive prefix over lanes
-__device__ __forceinline__ uint64_t warp_excl_u64(uint64_t v, int lane) {
-  uint64_t inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint64_t t = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += t;
+// A team of W warps (32 W threads) selects one plan row.  Thread t holds the
+// contiguous blocks [t VPL, (t+1) VPL) of the row in registers (VPL odd, so
+// the threads' blocked reads of the staged row hit distinct banks); every
+// cross-thread step is a warp shuffle plus, for W = 2, one exchange through
+// shared memory behind the team's named barrier.
+template <int W>
+struct Team {
+  uint64_t* red;    // W * 8 scratch words, used round-robin
+  uint32_t bar_id;  // named barrier of the team (W = 2)
+  int t, lane, wi;
+  uint32_t slot;
+  __device__ __forceinline__ void sync() const {
+    if constexpr (W == 1)
+      __syncwarp();
+    else
+      isa_dev::named_bar_sync(bar_id, 32 * W);
   }
-  return inc - v;
-}
-__device__ __forceinline__ uint32_t warp_excl_u32(uint32_t v, int lane) {
-  uint32_t inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += t;
+  // the other warp's value of a warp-uniform quantity (W = 2)
+  __device__ __forceinline__ uint64_t swap(uint64_t v) {
+    uint64_t* r = red + (slot++ & 7u) * W;
+    if (lane == 0) r[wi] = v;
+    sync();
+    return r[wi ^ 1];
   }
-  return inc - v;
-}
+  __device__ __forceinline__ uint64_t sum_u64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if constexpr (W == 1) return v;
+    return v + swap(v);
+  }
+  __device__ __forceinline__ uint32_t sum_u32(uint32_t v) {
+    v = __reduce_add_sync(0xffffffffu, v);
+    if constexpr (W == 1) return v;
+    return v + static_cast<uint32_t>(swap(v));
+  }
+  __device__ __forceinline__ uint32_t max_u32(uint32_t v) {
+    v = __reduce_max_sync(0xffffffffu, v);
+    if constexpr (W == 1) return v;
+    return max(v, static_cast<uint32_t>(swap(v)));
+  }
+  // exclusive prefix over the team's threads in order
+  __device__ __forceinline__ uint64_t excl_u64(uint64_t v) {
+    uint64_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t x = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += x;
+    }
+    if constexpr (W == 1) return inc - v;
+    const uint64_t other = swap(__shfl_sync(0xffffffffu, inc, 31));
+    return inc - v + (wi ? other : 0ull);
+  }
+};
 
-// One plan row by one warp.  st: the row's mass as staged by the caller
-// (element i at i + i / 32, so that the lanes' blocked reads are free of bank
-// conflicts), reused for the log-weight list once the keys are in registers;
-// hist: the warp's 256-bin radix histogram.
-template <int VPL>
-__device__ __forceinline__ void select_row_warp(const SelectLaunch& a, const int64_t row, uint32_t* st,
-                                                uint32_t* hist, const int lane) {
+// One plan row.  st: the row's mass as staged by the caller (element i at
+// st[i]), reused for the log-weight list once the keys are in registers;
+// hist: the team's 256-bin radix histogram.
+template <int VPL, int W>
+__device__ __forceinline__ void select_row_team(const SelectLaunch& a, const int64_t row, uint32_t* st,
+                                                uint32_t* hist, Team<W>& tm) {
+  static_assert(VPL <= 64, "flags are 64-bit masks");
   const int nK = a.nK;
-  auto at = [](int i) { return i + (i >> 5); };
+  const int t = tm.t, lane = tm.lane;
   const int g = static_cast<int>(row % a.G);
   const int h = static_cast<int>((row / a.G) % a.H);
   const int b = static_cast<int>(row / (static_cast<int64_t>(a.G) * a.H));
-  const int base = lane * VPL;
-  const int nv = max(0, min(VPL, nK - base));  // blocks this lane holds
+  const int base = t * VPL;
+  const int nv = max(0, min(VPL, nK - base));  // blocks this thread holds
   uint32_t key[VPL];
   bool bad = false;
 #pragma unroll
   for (int v = 0; v < VPL; ++v) {
     uint32_t k = 0;
     if (v < nv) {
-      const float x = __uint_as_float(st[at(base + v)]);
+      const float x = __uint_as_float(st[base + v]);
       if (!isfinite(x)) {
         bad = true;
       } else if (x > 0.0f) {
@@ -430,31 +459,37 @@ __device__ __forceinline__ void select_row_warp(const SelectLaunch& a, const int
   // ---- exact set: threshold t = largest key with #{key >= t} >= n_exact
   uint64_t ex = 0;  // bit v: block base+v is exact
   if (n_exact > 0) {
-    // t = the n_exact-th largest key, by a radix select over the key bytes
-    // from the top: a 256-bin histogram of the keys that match the prefix
-    // so far, and the bin holding the remaining rank (lane l owns bins
-    // 8l .. 8l+7, so the bins above a lane's are those of higher lanes)
-    uint32_t t = 0, mask = 0, kk = static_cast<uint32_t>(n_exact);
+    // the n_exact-th largest key, by a radix select over the key bytes from
+    // the top: a 256-bin histogram of the keys that match the prefix so far,
+    // and the bin holding the remaining rank (thread t owns bins
+    // BPT t .. BPT t + BPT - 1, so the bins above a thread's are those of
+    // higher threads)
+    constexpr int BPT = 256 / (32 * W);
+    uint32_t thr = 0, mask = 0, kk = static_cast<uint32_t>(n_exact);
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0u;
-      __syncwarp();
+      for (int i = 0; i < BPT; ++i) hist[t * BPT + i] = 0u;
+      tm.sync();
 #pragma unroll
       for (int v = 0; v < VPL; ++v)
-        if (v < nv && (key[v] & mask) == t) atomicAdd(&hist[(key[v] >> shift) & 255u], 1u);
-      __syncwarp();
-      uint32_t cnt[8], local = 0;
+        if (v < nv && (key[v] & mask) == thr) atomicAdd(&hist[(key[v] >> shift) & 255u], 1u);
+      tm.sync();
+      uint32_t cnt[BPT], local = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        cnt[i] = hist[lane * 8 + i];
+      for (int i = 0; i < BPT; ++i) {
+        cnt[i] = hist[t * BPT + i];
         local += cnt[i];
       }
-      uint32_t suf = local;  // keys in the bins of lanes >= this one
+      uint32_t suf = local;  // keys in the bins of threads >= this one (this warp)
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t x = __shfl_down_sync(0xffffffffu, suf, o);
         if (lane + o < 32) suf += x;
+      }
+      if constexpr (W == 2) {
+        const uint32_t up = static_cast<uint32_t>(tm.swap(__shfl_sync(0xffffffffu, suf, 0)));
+        if (tm.wi == 0) suf += up;  // the upper warp's bins are all above
       }
       const uint32_t above = suf - local;
       const bool here = above < kk && suf >= kk;
@@ -462,41 +497,44 @@ __device__ __forceinline__ void select_row_warp(const SelectLaunch& a, const int
       if (here) {
         uint32_t acc = above;
 #pragma unroll
-        for (int i = 7; i >= 0; --i) {
+        for (int i = BPT - 1; i >= 0; --i) {
           if (rem == 0 && acc + cnt[i] >= kk) {
-            sel = 8 * lane + i;
+            sel = BPT * t + i;
             rem = kk - acc;
           }
           acc += cnt[i];
         }
       }
-      const int src = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
-      sel = __shfl_sync(0xffffffffu, sel, src);
-      rem = __shfl_sync(0xffffffffu, rem, src);
-      t |= sel << shift;
+      // exactly one thread of the team holds the bin: share it
+      uint64_t pick = here ? ((static_cast<uint64_t>(sel) << 32) | rem) : 0ull;
+      const uint32_t src = __ballot_sync(0xffffffffu, here);
+      pick = src ? __shfl_sync(0xffffffffu, pick, __ffs(src) - 1) : 0ull;
+      if constexpr (W == 2) pick |= tm.swap(pick);  // the warp without it contributes 0
+      sel = static_cast<uint32_t>(pick >> 32);
+      rem = static_cast<uint32_t>(pick);
+      thr |= sel << shift;
       mask |= 255u << shift;
       kk = rem;
-      __syncwarp();  // every lane has read the histogram before it is cleared
     }
     uint32_t gt = 0, eq = 0;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
-      gt += (v < nv && key[v] > t) ? 1u : 0u;
-      eq += (v < nv && key[v] == t) ? 1u : 0u;
+      gt += (v < nv && key[v] > thr) ? 1u : 0u;
+      eq += (v < nv && key[v] == thr) ? 1u : 0u;
     }
-    const uint32_t need = static_cast<uint32_t>(n_exact) - __reduce_add_sync(0xffffffffu, gt);
-    uint32_t rank = warp_excl_u32(eq, lane);
+    const uint32_t need = static_cast<uint32_t>(n_exact) - tm.sum_u32(gt);
+    uint32_t rank = static_cast<uint32_t>(tm.excl_u64(eq));
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       if (v < nv) {
-        const bool tie = key[v] == t;
-        if (key[v] > t || (tie && rank < need)) ex |= 1ull << v;
+        const bool tie = key[v] == thr;
+        if (key[v] > thr || (tie && rank < need)) ex |= 1ull << v;
         rank += tie ? 1u : 0u;
       }
     }
   }
   // ---- the rest: weights (in registers, in place of the keys), capping,
-  // systematic PPS.  Every loop over the lane's blocks is unrolled, so the
+  // systematic PPS.  Every loop over the thread's blocks is unrolled, so the
   // per-block flags are bits at constant positions.
   const int n_rest = nK - n_exact;
   uint64_t cap = 0, drawn = 0;  // bit v: capped (or taken whole), drawn
@@ -511,7 +549,7 @@ __device__ __forceinline__ void select_row_warp(const SelectLaunch& a, const int
 #pragma unroll
     for (int v = 0; v < VPL; ++v)
       if (v < nv && !((ex >> v) & 1)) kmax = max(kmax, key[v]);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    kmax = tm.max_u32(kmax);
     const double mmax = static_cast<double>(__uint_as_float(kmax));
     const double c31 = mmax > 0.0 ? 2147483648.0 / mmax : 0.0;
     // w = floor(m / m_max * 2^31) + 1 on the rest; 0 on the exact set and past the row
@@ -522,13 +560,13 @@ __device__ __forceinline__ void select_row_warp(const SelectLaunch& a, const int
       key[v] = wv;
     }
     int n_capped = 0;
-    uint64_t tl = 0;  // after the loop: this lane's total over the uncapped rest
+    uint64_t tl = 0;  // after the loop: this thread's total over the uncapped rest
     for (;;) {
       tl = 0;
 #pragma unroll
       for (int v = 0; v < VPL; ++v)
         if (!((cap >> v) & 1)) tl += key[v];
-      T = warp_sum_u64(tl);
+      T = tm.sum_u64(tl);
       n_left = n_sample - n_capped;
       uint32_t add = 0;
       uint64_t newcap = 0;
@@ -539,7 +577,7 @@ __device__ __forceinline__ void select_row_warp(const SelectLaunch& a, const int
           ++add;
         }
       }
-      const uint32_t add_all = __reduce_add_sync(0xffffffffu, add);
+      const uint32_t add_all = tm.sum_u32(add);
       if (add_all == 0) break;
       cap |= newcap;
       n_capped += static_cast<int>(add_all);
@@ -553,10 +591,10 @@ __device__ __forceinline__ void select_row_warp(const SelectLaunch& a, const int
       // points of the comb below x: q + [r 2^32 > U T] with q = floor(x n' / T)
       // and r = x n' - q T; r 2^32 > U T is r > floor(U T / 2^32) for whole r.
       // Walking x up by an uncapped weight (n' w < T) moves r up by n' w and
-      // needs at most one reduction by T, so only the start of each lane's
+      // needs at most one reduction by T, so only the start of each thread's
       // segment takes a division.
       const uint64_t thr = static_cast<uint64_t>(U) * (T >> 32) + ((static_cast<uint64_t>(U) * (T & 0xFFFFFFFFull)) >> 32);
-      const uint64_t xn0 = warp_excl_u64(tl, lane) * nl;
+      const uint64_t xn0 = tm.excl_u64(tl) * nl;
       uint64_t r = xn0 % T;
       uint32_t q = static_cast<uint32_t>(xn0 / T);  // at most n'
       uint32_t f_prev = q + (r > thr ? 1u : 0u);
@@ -577,16 +615,17 @@ __device__ __forceinline__ void select_row_warp(const SelectLaunch& a, const int
   }
   // ---- write the plan row: exact ascending, then capped + drawn ascending.
   // The drawn blocks' log-weights are left to a second, converged pass over
-  // the rest part of the row: each lane records, per rest position it fills,
-  // the drawn block's weight (0 for a capped block) in the warp's shared
-  // slice, which no longer holds anything the warp reads.
+  // the rest part of the row: each thread records, per rest position it
+  // fills, the drawn block's weight (0 for a capped block) in the team's
+  // staged row, which no longer holds anything the team reads.
   int32_t* out_idx = a.idx + row * S;
   float* out_lw = a.log_w + row * S;
   const int n_rs = S - n_exact;
   const uint32_t ne = __popcll(ex), nr = __popcll(cap | drawn);
-  uint32_t pe = warp_excl_u32(ne, lane);
-  uint32_t pr = warp_excl_u32(nr, lane);
-  __syncwarp();
+  const uint64_t pre = tm.excl_u64((static_cast<uint64_t>(ne) << 32) | nr);  // both counts < 2^32
+  uint32_t pe = static_cast<uint32_t>(pre >> 32);
+  uint32_t pr = static_cast<uint32_t>(pre);
+  tm.sync();
 #pragma unroll
   for (int v = 0; v < VPL; ++v) {
     const int i = base + v;
@@ -604,17 +643,17 @@ __device__ __forceinline__ void select_row_warp(const SelectLaunch& a, const int
       ++pr;
     }
   }
-  __syncwarp();
-  const uint32_t tot_e = __reduce_add_sync(0xffffffffu, ne), tot_r = __reduce_add_sync(0xffffffffu, nr);
+  const uint64_t tot = tm.sum_u64((static_cast<uint64_t>(ne) << 32) | nr);  // also orders the list writes
+  const uint32_t tot_e = static_cast<uint32_t>(tot >> 32), tot_r = static_cast<uint32_t>(tot);
   const double lnT = T > 0 ? log(static_cast<double>(T)) : 0.0;
   const int n_w = min(static_cast<int>(tot_r), n_rs);
-  for (int k = lane; k < n_w; k += 32) {
+  for (int k = t; k < n_w; k += 32 * W) {
     const uint32_t wv = st[k];
     out_lw[n_exact + k] =
         wv ? static_cast<float>(lnT - log(static_cast<double>(static_cast<uint64_t>(n_left) * wv))) : 0.0f;
   }
-  const bool any_bad = __any_sync(0xffffffffu, bad);
-  if (lane == 0 && (any_bad || tot_e != static_cast<uint32_t>(n_exact) || tot_e + tot_r != static_cast<uint32_t>(S)))
+  const uint32_t any_bad = tm.sum_u32(bad ? 1u : 0u);
+  if (t == 0 && (any_bad || tot_e != static_cast<uint32_t>(n_exact) || tot_e + tot_r != static_cast<uint32_t>(S)))
     atomicCAS(a.status, 0, kStatusDeviceCheck);
 }
 
@@ -622,22 +661,41 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 
-// Persistent warps: warp w of the grid takes rows w, w + W, w + 2W, ... (W =
-// the grid's warps) and stages the next row's mass in its second shared
-// buffer (cp.async) while it selects the current one.
+// Persistent teams of two warps: team w of the grid takes rows w, w + W,
+// w + 2W, ... (W = the grid's teams) and stages the next row's mass in its
+// second shared buffer (cp.async) while it selects the current one.
+constexpr int kTeamWarps = 2;
+constexpr int kTeamsPerCta = kWarpRowsPerCta / kTeamWarps;
+
 template <int VPL>
-__global__ void __launch_bounds__(32 * kWarpRowsPerCta, VPL <= 40 ? 2 : 1) select_warp_kernel(SelectLaunch a) {
+struct TeamLayout {
+  static constexpr int kSlice = 32 * kTeamWarps * VPL;  // one staged row
+  static constexpr int kTeamWords = 2 * kSlice + 256 + 2 * 8 * kTeamWarps;  // two rows, histogram, scratch
+  static constexpr size_t kBytes = static_cast<size_t>(kTeamsPerCta) * kTeamWords * 4;
+};
+
+template <int VPL>
+__global__ void __launch_bounds__(32 * kWarpRowsPerCta, VPL <= 19 ? 3 : 1) select_team_kernel(SelectLaunch a) {
+  using L = TeamLayout<VPL>;
   extern __shared__ __align__(16) uint8_t sm[];
-  constexpr int kSlice = 32 * VPL + VPL;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int team = warp / kTeamWarps;
   const int64_t rows = static_cast<int64_t>(a.B) * a.H * a.G;
-  uint32_t* st = reinterpret_cast<uint32_t*>(sm) + warp * 2 * kSlice;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(sm) + kWarpRowsPerCta * 2 * kSlice + warp * 256;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarpRowsPerCta;
-  int64_t row = static_cast<int64_t>(blockIdx.x) * kWarpRowsPerCta + warp;
+  uint32_t* tw = reinterpret_cast<uint32_t*>(sm) + team * L::kTeamWords;
+  uint32_t* st = tw;
+  uint32_t* hist = tw + 2 * L::kSlice;
+  Team<kTeamWarps> tm;
+  tm.red = reinterpret_cast<uint64_t*>(hist + 256);
+  tm.bar_id = 1u + static_cast<uint32_t>(team);
+  tm.t = threadIdx.x - team * 32 * kTeamWarps;
+  tm.lane = threadIdx.x & 31;
+  tm.wi = warp % kTeamWarps;
+  tm.slot = 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kTeamsPerCta;
+  int64_t row = static_cast<int64_t>(blockIdx.x) * kTeamsPerCta + team;
   auto stage = [&](int64_t r, uint32_t* dst) {
     const float* m = a.mass + r * a.nK;
-    for (int i = lane; i < a.nK; i += 32) cp_async4(isa_dev::smem_addr(dst + i + (i >> 5)), m + i);
+    for (int i = tm.t; i < a.nK; i += 32 * kTeamWarps) cp_async4(isa_dev::smem_addr(dst + i), m + i);
   };
   using isa_dev::cp_async_commit;
   using isa_dev::cp_async_wait_group;
@@ -645,13 +703,13 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, VPL <= 40 ? 2 : 1) selec
   cp_async_commit();
   int buf = 0;
   for (; row < rows; row += stride) {
-    if (row + stride < rows) stage(row + stride, st + (buf ^ 1) * kSlice);
+    if (row + stride < rows) stage(row + stride, st + (buf ^ 1) * L::kSlice);
     cp_async_commit();
-    cp_async_wait_group<1>();  // this lane's copies of the current row have landed
-    __syncwarp();
-    if (a.discard_mass) discard_row_lines(a.mass + row * a.nK, a.nK, lane, 32);
-    select_row_warp<VPL>(a, row, st + buf * kSlice, hist, lane);
-    __syncwarp();  // the buffer is restaged only after every lane is done with it
+    cp_async_wait_group<1>();  // this thread's copies of the current row have landed
+    tm.sync();
+    if (a.discard_mass) discard_row_lines(a.mass + row * a.nK, a.nK, tm.t, 32 * kTeamWarps);
+    select_row_team<VPL, kTeamWarps>(a, row, st + buf * L::kSlice, hist, tm);
+    tm.sync();  // the buffer is restaged only after every thread is done with it
     buf ^= 1;
   }
   cp_async_wait_group<0>();
@@ -740,22 +798,23 @@ __global__ void __launch_bounds__(kSelThreads) top_p_count_kernel(const float* _
 }
 
 template <int VPL>
-int launch_select_warp(const SelectLaunch& s, cudaStream_t stream) {
+int launch_select_team(const SelectLaunch& s, cudaStream_t stream) {
+  using L = TeamLayout<VPL>;
   const long long rows = static_cast<long long>(s.B) * s.H * s.G;
-  const size_t smem = static_cast<size_t>(kWarpRowsPerCta) * (2 * (32 * VPL + VPL) + 256) * 4;
+  const size_t smem = L::kBytes;
   if (smem > 48 * 1024) {
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_warp_kernel<VPL>), static_cast<int>(smem));
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_team_kernel<VPL>), static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
   }
   int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_warp_kernel<VPL>,
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_team_kernel<VPL>,
                                                                 32 * kWarpRowsPerCta, smem);
   if (e != cudaSuccess) return static_cast<int>(e);
   if (per_sm < 1) return static_cast<int>(cudaErrorInvalidConfiguration);
-  const long long want = (rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta;
+  const long long want = (rows + kTeamsPerCta - 1) / kTeamsPerCta;
   const long long cap = static_cast<long long>(s.num_sms > 0 ? s.num_sms : 148) * per_sm;
   const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
-  select_warp_kernel<VPL><<<grid, 32 * kWarpRowsPerCta, smem, stream>>>(s);
+  select_team_kernel<VPL><<<grid, 32 * kWarpRowsPerCta, smem, stream>>>(s);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -773,10 +832,11 @@ int launch_top_p_count(const float* mass, int rows, int nK, double top_p, int S,
 }
 
 int launch_select(const SelectLaunch& s, cudaStream_t stream) {
-  if (s.nK <= 32 * 8) return launch_select_warp<8>(s, stream);
-  if (s.nK <= 32 * 16) return launch_select_warp<16>(s, stream);
-  if (s.nK <= 32 * 40) return launch_select_warp<40>(s, stream);
-  if (s.nK <= 32 * 64) return launch_select_warp<64>(s, stream);
+  constexpr int TT = 32 * kTeamWarps;  // threads per team
+  if (s.nK <= TT * 5) return launch_select_team<5>(s, stream);
+  if (s.nK <= TT * 9) return launch_select_team<9>(s, stream);
+  if (s.nK <= TT * 19) return launch_select_team<19>(s, stream);
+  if (s.nK <= TT * 33) return launch_select_team<33>(s, stream);
   const size_t smem = static_cast<size_t>(s.nK) * 9 + 16;
   if (smem > 48 * 1024) {
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel), static_cast<int>(smem));
