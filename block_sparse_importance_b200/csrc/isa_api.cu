@@ -321,9 +321,11 @@ isa_status do_pipeline(isa_context* ctx, const isa_shape* s, const isa_params* p
   return do_attention(ctx, s, q, k, v, idx, lw, static_cast<int32_t>(S), out, lse, aws, attn_ws_bytes(s), false, st);
 }
 
-// isa_plan: heads per chunk, so that one chunk's mass stays well inside L2
-// between the mass kernel that writes it and the selector that reads it.
-constexpr size_t kPlanChunkMassBytes = size_t(48) << 20;
+// isa_plan: heads per chunk, so that one chunk's mass stays inside L2 (126 MB)
+// between the mass kernel that writes it and the selector that reads it,
+// while a chunk still gives the kernels enough CTAs to fill the SMs (at the
+// Hunyuan shape one head's mass is 28 MB and fills under half the SMs).
+constexpr size_t kPlanChunkMassBytes = size_t(88) << 20;
 
 int plan_chunk_heads(const isa_shape* s) {
   const size_t per_head = static_cast<size_t>(s->num_groups) * nblocks(s) * 4;

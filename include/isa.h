@@ -295,7 +295,7 @@ ISA_API isa_status isa_dense_attention(isa_context* ctx, const isa_shape* shape,
  * sampler directly; plans are made from the current activations and may then
  * serve several attention calls).  The result equals isa_select(isa_score(.))
  * bit for bit, but the estimated mass never reaches HBM: the layer is
- * scored and selected in chunks of heads whose mass (at most 48 MiB, at
+ * scored and selected in chunks of heads whose mass (at most 88 MiB, at
  * least one head) stays in L2 between the two steps, and the selector drops
  * every mass line it has read from L2 without writing it back.  The
  * workspace (isa_plan_workspace_bytes, 256-byte aligned) holds one chunk's
