@@ -392,9 +392,10 @@ struct KtLayout {
   static constexpr uint32_t kOhBytes = 2 * kNGroup;             // 16 cluster slots
   static constexpr uint32_t kMc = kKtSlots * kXBytes;
   static constexpr uint32_t kOh = kMc + kKtSets * kMcBytes;
-  // per set: |mu|^2 partials [16][4], |mu|^2 [16], counts [16], reciprocal counts [16]
+  // per set: |mu|^2 partials [16][4], |mu|^2 [16], counts [16], reciprocal
+  // counts [16], count partials [16][4]
   static constexpr uint32_t kRed = kOh + kKtSets * kOhBytes;
-  static constexpr uint32_t kRedBytes = (64 + 16 + 16 + 16) * 4;
+  static constexpr uint32_t kRedBytes = (64 + 16 + 16 + 16 + 64) * 4;
   static constexpr uint32_t kBar = kRed + kKtSets * kRedBytes;
   static constexpr int kXFull = 0, kXEmpty = kKtSlots, kMmaDone = 2 * kKtSlots, kNumBars = 2 * kKtSlots + kKtSets;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // TMEM address, abort flag; released[] at +16
@@ -550,6 +551,7 @@ __global__ void __launch_bounds__(kKtThreads, 1)
     float* nsq_fin = nsq_part + 64;                                                // [16]
     uint32_t* cnt = reinterpret_cast<uint32_t*>(nsq_fin + 16);                      // [16]
     float* inv = reinterpret_cast<float*>(cnt + 16);                               // [16]
+    uint32_t* cnt_part = reinterpret_cast<uint32_t*>(inv + 16);                    // [16][4]
     constexpr uint32_t idesc_assign = idesc_bf16_f32(128, 2 * CP, 1, 0);
     constexpr uint32_t idesc_update = idesc_bf16_f32(128, 16, 1, 1);
     uint32_t mma_waits = 0;
@@ -665,7 +667,6 @@ __global__ void __launch_bounds__(kKtThreads, 1)
         } else if (q4 == q_aux && lane < CP) {
           const float4 np = *reinterpret_cast<const float4*>(nsq_part + 4 * lane);
           nsq_fin[lane] = (np.x + np.y) + (np.z + np.w);
-          cnt[lane] = 0u;
         }
         pending = true;
         if (!wait_mma()) {
@@ -715,11 +716,12 @@ __global__ void __launch_bounds__(kKtThreads, 1)
             oh_row[j * (L::kNGroup / 16)] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
           }
         }
+        // this warp's count of each cluster: one ballot per cluster
 #pragma unroll
         for (int c = 0; c < CP; ++c) {
           if (c < C) {
             const uint32_t b = __ballot_sync(0xffffffffu, label == c);
-            if (lane == 0 && b) atomicAdd(&cnt[c], static_cast<uint32_t>(__popc(b)));
+            if (lane == 0) cnt_part[c * 4 + q4] = static_cast<uint32_t>(__popc(b));
           }
         }
         fence_proxy_async_smem();
@@ -735,7 +737,9 @@ __global__ void __launch_bounds__(kKtThreads, 1)
               mma_ss(tmem + col_u, da + ((kk * 2048) >> 4), db + ((kk * 256) >> 4), idesc_update, kk > 0 ? 1u : 0u);
           if (elect_one()) tc_commit(bar(L::kMmaDone + s));
         } else if (q4 == q_aux && lane < CP) {
-          const uint32_t cc = cnt[lane];
+          const uint4 cp4 = *reinterpret_cast<const uint4*>(cnt_part + 4 * lane);
+          const uint32_t cc = lane < C ? (cp4.x + cp4.y) + (cp4.z + cp4.w) : 0u;
+          cnt[lane] = cc;
           inv[lane] = cc > 0u ? 1.0f / static_cast<float>(cc) : 0.0f;
         }
         pending = true;
@@ -845,20 +849,64 @@ __global__ void __launch_bounds__(kMassThreads, 1)
   const int T = (nK + 127) / 128;
   const int n_items = 2 * T;
 
+  // The producer thread sets up the barriers and starts the first k-bar tiles
+  // on their way before the centroid conversion below: they do not depend on
+  // it, and the other threads touch no barrier before the block-wide sync.
+  auto load_item = [&](int i) {
+    const uint32_t slot = i % kMassRing;
+    mbar_arrive_expect_tx(bar(L::kBarFull + slot), L::kStage);
+    const uint32_t dst = base + L::kRing + slot * L::kStage;
+    const int row = (i % T) * 128;
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(dst + c * L::kChunk, &tm_hi, bar(L::kBarFull + slot), c * 64, row, static_cast<int>(bh));
+      tma_load_3d(dst + L::kTile + c * L::kChunk, &tm_lo, bar(L::kBarFull + slot), c * 64, row,
+                  static_cast<int>(bh));
+    }
+  };
+  const int pre = n_items < kMassRing ? n_items : kMassRing;  // loads issued before the sync
+  if (warp == kProducer && lane == 0) {
+    for (int i = 0; i < kMassRing; ++i) {
+      mbar_init(bar(L::kBarFull + i), 1);
+      mbar_init(bar(L::kBarEmpty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::kBarSFull + i), 1);
+      mbar_init(bar(L::kBarSFree + i), kMassSoftmaxWarps * 32);
+    }
+    mbar_init(bar(L::kBarFinal), 1);
+    mbar_init(bar(L::kBarXchg), kMassSoftmaxWarps * 32);
+    *abort_flag = 0;
+    fence_mbar_init();
+    for (int i = 0; i < pre; ++i) load_item(i);
+  }
   // centroid rows -> bf16 hi / lo, K-major with the 128-byte swizzle (16-byte
-  // granule q of row r stored at granule q ^ (r & 7) of the row)
-  for (int i = tid; i < 128 * (D / 8); i += kMassThreads) {
+  // granule q of row r stored at granule q ^ (r & 7) of the row).  Each thread
+  // issues the loads of all its granules before it converts any, so that
+  // the global-memory latency is paid once.
+  constexpr int kPer = (128 * (D / 8) + kMassThreads - 1) / kMassThreads;
+  float4 ld[kPer][2];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = tid + u * kMassThreads;
     const int r = i / (D / 8), q = i - r * (D / 8);
     const int gl = r / Cp, c = r - gl * Cp, g = g0 + gl;
-    float v[8];
-    if (c < C && g < G) {
+    if (i < 128 * (D / 8) && c < C && g < G) {
       const float4* src = reinterpret_cast<const float4*>(centroids + ((bh * G + g) * C + c) * D + q * 8);
-      const float4 x0 = src[0], x1 = src[1];
-      v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w; v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+      ld[u][0] = src[0];
+      ld[u][1] = src[1];
     } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+      ld[u][0] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      ld[u][1] = ld[u][0];
     }
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = tid + u * kMassThreads;
+    if (i >= 128 * (D / 8)) break;
+    const int r = i / (D / 8), q = i - r * (D / 8);
+    const float v[8] = {ld[u][0].x, ld[u][0].y, ld[u][0].z, ld[u][0].w,
+                        ld[u][1].x, ld[u][1].y, ld[u][1].z, ld[u][1].w};
     uint32_t hi[4], lo[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -873,20 +921,6 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     *reinterpret_cast<uint4*>(smem + L::kAHi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(smem + L::kALo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
-  if (tid == 0) {
-    for (int i = 0; i < kMassRing; ++i) {
-      mbar_init(bar(L::kBarFull + i), 1);
-      mbar_init(bar(L::kBarEmpty + i), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(L::kBarSFull + i), 1);
-      mbar_init(bar(L::kBarSFree + i), kMassSoftmaxWarps * 32);
-    }
-    mbar_init(bar(L::kBarFinal), 1);
-    mbar_init(bar(L::kBarXchg), kMassSoftmaxWarps * 32);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
   if (warp == kMma) {
     tmem_alloc(smem_addr(tmem_slot), 256);
     tmem_relinquish();
@@ -900,24 +934,16 @@ __global__ void __launch_bounds__(kMassThreads, 1)
 
   if (warp == kProducer) {
     // ------------------------------------------------------------ producer
-    uint32_t issued = 0;
+    uint32_t issued = static_cast<uint32_t>(pre);
     bool ok = true;
     if (lane == 0) {
-      for (int i = 0; i < n_items && ok; ++i) {
+      for (int i = pre; i < n_items && ok; ++i) {
         const uint32_t slot = i % kMassRing, use = i / kMassRing;
         if (!mbar_wait(bar(L::kBarEmpty + slot), (use & 1u) ^ 1u, abort_flag, kWaitTimeoutNs)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(L::kBarFull + slot), L::kStage);
-        const uint32_t dst = base + L::kRing + slot * L::kStage;
-        const int row = (i % T) * 128;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(dst + c * L::kChunk, &tm_hi, bar(L::kBarFull + slot), c * 64, row, static_cast<int>(bh));
-          tma_load_3d(dst + L::kTile + c * L::kChunk, &tm_lo, bar(L::kBarFull + slot), c * 64, row,
-                      static_cast<int>(bh));
-        }
+        load_item(i);
         ++issued;
       }
       if (!ok || *abort_flag) {
