@@ -425,11 +425,16 @@ struct Team {
 
 // One plan row.  st: the row's mass as staged by the caller (element i at
 // st[i]), reused for the log-weight list once the keys are in registers;
-// hist: the team's 256-bin radix histogram.
+// hist: the team's 256-bin radix histogram; scr: VPL words of this thread's
+// scratch (the drawn blocks' weights, in block order).  The passes over the
+// thread's blocks are fused where the data allow: the first radix round with
+// the key extraction, the exact set with the rest's maximum, the weights with
+// their sum; the capping pass runs only when a weight can reach the cap.
 template <int VPL, int W>
 __device__ __forceinline__ void select_row_team(const SelectLaunch& a, const int64_t row, uint32_t* st,
-                                                uint32_t* hist, Team<W>& tm) {
+                                                uint32_t* hist, uint32_t* scr, Team<W>& tm) {
   static_assert(VPL <= 64, "flags are 64-bit masks");
+  constexpr int BPT = 256 / (32 * W);  // histogram bins owned by each thread
   const int nK = a.nK;
   const int t = tm.t, lane = tm.lane;
   const int g = static_cast<int>(row % a.G);
@@ -437,6 +442,17 @@ __device__ __forceinline__ void select_row_team(const SelectLaunch& a, const int
   const int b = static_cast<int>(row / (static_cast<int64_t>(a.G) * a.H));
   const int base = t * VPL;
   const int nv = max(0, min(VPL, nK - base));  // blocks this thread holds
+  const int S = a.n_exact + a.n_sample;
+  // the row's split of the plan: fixed, or per row (top-p rule)
+  const int n_exact = a.ne_rows ? min(max(a.ne_rows[row], 0), S) : a.n_exact;
+  const int n_sample = S - n_exact;
+  if (n_exact > 0) {
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) hist[t * BPT + i] = 0u;
+    tm.sync();
+  }
+  // ---- keys (mass bits; 0 for non-positive, non-finite or past the row),
+  // with the first radix round's histogram of their top byte
   uint32_t key[VPL];
   bool bad = false;
 #pragma unroll
@@ -449,31 +465,29 @@ __device__ __forceinline__ void select_row_team(const SelectLaunch& a, const int
       } else if (x > 0.0f) {
         k = __float_as_uint(x);
       }
+      if (n_exact > 0) atomicAdd(&hist[k >> 24], 1u);
     }
-    key[v] = k;  // blocks past the row are 0 and never counted (v >= nv)
+    key[v] = k;
   }
-  const int S = a.n_exact + a.n_sample;
-  // the row's split of the plan: fixed, or per row (top-p rule)
-  const int n_exact = a.ne_rows ? min(max(a.ne_rows[row], 0), S) : a.n_exact;
-  const int n_sample = S - n_exact;
-  // ---- exact set: threshold t = largest key with #{key >= t} >= n_exact
-  uint64_t ex = 0;  // bit v: block base+v is exact
+  // ---- exact set: the n_exact largest keys, ties to the lower block
+  uint64_t ex = 0;    // bit v: block base+v is exact
+  uint32_t kmax = 0;  // the largest key of the rest
   if (n_exact > 0) {
-    // the n_exact-th largest key, by a radix select over the key bytes from
-    // the top: a 256-bin histogram of the keys that match the prefix so far,
-    // and the bin holding the remaining rank (thread t owns bins
-    // BPT t .. BPT t + BPT - 1, so the bins above a thread's are those of
-    // higher threads)
-    constexpr int BPT = 256 / (32 * W);
+    // the n_exact-th largest key thr, by a radix select over the key bytes
+    // from the top: a histogram of the keys that match the prefix so far, and
+    // the bin holding the remaining rank (thread t owns bins BPT t ..
+    // BPT t + BPT - 1, so the bins above a thread's are those of higher threads)
     uint32_t thr = 0, mask = 0, kk = static_cast<uint32_t>(n_exact);
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
+      if (shift < 24) {
 #pragma unroll
-      for (int i = 0; i < BPT; ++i) hist[t * BPT + i] = 0u;
-      tm.sync();
+        for (int i = 0; i < BPT; ++i) hist[t * BPT + i] = 0u;
+        tm.sync();
 #pragma unroll
-      for (int v = 0; v < VPL; ++v)
-        if (v < nv && (key[v] & mask) == thr) atomicAdd(&hist[(key[v] >> shift) & 255u], 1u);
+        for (int v = 0; v < VPL; ++v)
+          if (v < nv && (key[v] & mask) == thr) atomicAdd(&hist[(key[v] >> shift) & 255u], 1u);
+      }
       tm.sync();
       uint32_t cnt[BPT], local = 0;
 #pragma unroll
@@ -515,23 +529,35 @@ __device__ __forceinline__ void select_row_team(const SelectLaunch& a, const int
       thr |= sel << shift;
       mask |= 255u << shift;
       kk = rem;
+      if constexpr (W == 1) tm.sync();  // every lane has read the histogram before it is cleared
     }
-    uint32_t gt = 0, eq = 0;
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-      gt += (v < nv && key[v] > thr) ? 1u : 0u;
-      eq += (v < nv && key[v] == thr) ? 1u : 0u;
-    }
-    const uint32_t need = static_cast<uint32_t>(n_exact) - tm.sum_u32(gt);
-    uint32_t rank = static_cast<uint32_t>(tm.excl_u64(eq));
+    // keys above thr are exact, and the lowest kk of the keys equal to thr
+    // (kk = n_exact - #{key > thr}); the rest's maximum is thr if a tie is
+    // left over, else the largest key below thr
+    uint64_t eqm = 0;
+    uint32_t below = 0;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       if (v < nv) {
-        const bool tie = key[v] == thr;
-        if (key[v] > thr || (tie && rank < need)) ex |= 1ull << v;
-        rank += tie ? 1u : 0u;
+        if (key[v] > thr) ex |= 1ull << v;
+        if (key[v] == thr) eqm |= 1ull << v;
+        if (key[v] < thr) below = max(below, key[v]);
       }
     }
+    uint32_t rank = static_cast<uint32_t>(tm.excl_u64(__popcll(eqm)));
+    bool tie_left = false;
+    for (uint64_t m = eqm; m; m &= m - 1) {
+      if (rank < kk)
+        ex |= m & (~m + 1);
+      else
+        tie_left = true;
+      ++rank;
+    }
+    kmax = tie_left ? thr : below;
+  } else {
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
+      if (v < nv) kmax = max(kmax, key[v]);
   }
   // ---- the rest: weights (in registers, in place of the keys), capping,
   // systematic PPS.  Every loop over the thread's blocks is unrolled, so the
@@ -545,42 +571,49 @@ __device__ __forceinline__ void select_row_team(const SelectLaunch& a, const int
     for (int v = 0; v < VPL; ++v)
       if (v < nv && !((ex >> v) & 1)) cap |= 1ull << v;
   } else if (n_sample > 0) {
-    uint32_t kmax = 0;
-#pragma unroll
-    for (int v = 0; v < VPL; ++v)
-      if (v < nv && !((ex >> v) & 1)) kmax = max(kmax, key[v]);
     kmax = tm.max_u32(kmax);
     const double mmax = static_cast<double>(__uint_as_float(kmax));
     const double c31 = mmax > 0.0 ? 2147483648.0 / mmax : 0.0;
-    // w = floor(m / m_max * 2^31) + 1 on the rest; 0 on the exact set and past the row
+    // w = floor(m / m_max * 2^31) + 1 on the rest; 0 on the exact set and past
+    // the row; with their sum and maximum
+    uint64_t tl = 0;
+    uint32_t wmax = 0;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       uint32_t wv = 0;
       if (v < nv && !((ex >> v) & 1)) wv = quant_weight(key[v], mmax, c31);
       key[v] = wv;
+      tl += wv;
+      wmax = max(wmax, wv);
     }
-    int n_capped = 0;
-    uint64_t tl = 0;  // after the loop: this thread's total over the uncapped rest
-    for (;;) {
-      tl = 0;
+    T = tm.sum_u64(tl);
+    n_left = n_sample;
+    // capping: repeat {T = sum of uncapped w, n' = n_s - #capped, cap every
+    // uncapped block with n' w >= T} until nothing changes; no block is capped
+    // when even the largest weight stays below T / n_s
+    if (static_cast<uint64_t>(n_sample) * tm.max_u32(wmax) >= T) {
+      int n_capped = 0;
+      for (;;) {
+        uint32_t add = 0;
+        uint64_t newcap = 0;
 #pragma unroll
-      for (int v = 0; v < VPL; ++v)
-        if (!((cap >> v) & 1)) tl += key[v];
-      T = tm.sum_u64(tl);
-      n_left = n_sample - n_capped;
-      uint32_t add = 0;
-      uint64_t newcap = 0;
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) {
-        if (key[v] != 0 && !((cap >> v) & 1) && static_cast<uint64_t>(n_left) * key[v] >= T) {
-          newcap |= 1ull << v;
-          ++add;
+        for (int v = 0; v < VPL; ++v) {
+          if (key[v] != 0 && !((cap >> v) & 1) && static_cast<uint64_t>(n_left) * key[v] >= T) {
+            newcap |= 1ull << v;
+            ++add;
+          }
         }
+        const uint32_t add_all = tm.sum_u32(add);
+        if (add_all == 0) break;
+        cap |= newcap;
+        n_capped += static_cast<int>(add_all);
+        tl = 0;
+#pragma unroll
+        for (int v = 0; v < VPL; ++v)
+          if (!((cap >> v) & 1)) tl += key[v];
+        T = tm.sum_u64(tl);
+        n_left = n_sample - n_capped;
       }
-      const uint32_t add_all = tm.sum_u32(add);
-      if (add_all == 0) break;
-      cap |= newcap;
-      n_capped += static_cast<int>(add_all);
     }
     if (n_left > 0) {
       const uint32_t U = static_cast<uint32_t>(
@@ -592,12 +625,14 @@ __device__ __forceinline__ void select_row_team(const SelectLaunch& a, const int
       // and r = x n' - q T; r 2^32 > U T is r > floor(U T / 2^32) for whole r.
       // Walking x up by an uncapped weight (n' w < T) moves r up by n' w and
       // needs at most one reduction by T, so only the start of each thread's
-      // segment takes a division.
+      // segment takes a division.  A drawn block's weight goes to the
+      // thread's scratch, in block order.
       const uint64_t thr = static_cast<uint64_t>(U) * (T >> 32) + ((static_cast<uint64_t>(U) * (T & 0xFFFFFFFFull)) >> 32);
       const uint64_t xn0 = tm.excl_u64(tl) * nl;
       uint64_t r = xn0 % T;
       uint32_t q = static_cast<uint32_t>(xn0 / T);  // at most n'
       uint32_t f_prev = q + (r > thr ? 1u : 0u);
+      int nd = 0;
 #pragma unroll
       for (int v = 0; v < VPL; ++v) {
         if (key[v] != 0 && !((cap >> v) & 1)) {
@@ -607,17 +642,21 @@ __device__ __forceinline__ void select_row_team(const SelectLaunch& a, const int
             ++q;
           }
           const uint32_t f = q + (r > thr ? 1u : 0u);
-          if (f != f_prev) drawn |= 1ull << v;
+          if (f != f_prev) {
+            drawn |= 1ull << v;
+            scr[nd++] = key[v];
+          }
           f_prev = f;
         }
       }
     }
   }
   // ---- write the plan row: exact ascending, then capped + drawn ascending.
-  // The drawn blocks' log-weights are left to a second, converged pass over
-  // the rest part of the row: each thread records, per rest position it
-  // fills, the drawn block's weight (0 for a capped block) in the team's
-  // staged row, which no longer holds anything the team reads.
+  // Each thread walks only its set flag bits.  The drawn blocks' log-weights
+  // are left to a second, converged pass over the rest part of the row: each
+  // thread records, per rest position it fills, the drawn block's weight (0
+  // for a capped block) in the team's staged row, which no longer holds
+  // anything the team reads.
   int32_t* out_idx = a.idx + row * S;
   float* out_lw = a.log_w + row * S;
   const int n_rs = S - n_exact;
@@ -626,21 +665,21 @@ __device__ __forceinline__ void select_row_team(const SelectLaunch& a, const int
   uint32_t pe = static_cast<uint32_t>(pre >> 32);
   uint32_t pr = static_cast<uint32_t>(pre);
   tm.sync();
-#pragma unroll
-  for (int v = 0; v < VPL; ++v) {
-    const int i = base + v;
-    if ((ex >> v) & 1) {
-      if (pe < static_cast<uint32_t>(n_exact)) {
-        out_idx[pe] = i;
-        out_lw[pe] = 0.0f;
-      }
-      ++pe;
-    } else if (((cap | drawn) >> v) & 1) {
-      if (pr < static_cast<uint32_t>(n_rs)) {
-        out_idx[n_exact + pr] = i;
-        st[pr] = ((drawn >> v) & 1) ? key[v] : 0u;
-      }
-      ++pr;
+  for (uint64_t m = ex; m; m &= m - 1, ++pe) {
+    if (pe < static_cast<uint32_t>(n_exact)) {
+      out_idx[pe] = base + __ffsll(static_cast<long long>(m)) - 1;
+      out_lw[pe] = 0.0f;
+    }
+  }
+  int jd = 0;
+  for (uint64_t m = cap | drawn; m; m &= m - 1, ++pr) {
+    const uint64_t bit = m & (~m + 1);
+    const bool is_drawn = (drawn & bit) != 0;
+    const uint32_t wv = is_drawn ? scr[jd] : 0u;
+    jd += is_drawn ? 1 : 0;
+    if (pr < static_cast<uint32_t>(n_rs)) {
+      out_idx[n_exact + pr] = base + __ffsll(static_cast<long long>(m)) - 1;
+      st[pr] = wv;
     }
   }
   const uint64_t tot = tm.sum_u64((static_cast<uint64_t>(ne) << 32) | nr);  // also orders the list writes
@@ -670,7 +709,8 @@ constexpr int kTeamsPerCta = kWarpRowsPerCta / kTeamWarps;
 template <int VPL>
 struct TeamLayout {
   static constexpr int kSlice = 32 * kTeamWarps * VPL;  // one staged row
-  static constexpr int kTeamWords = 2 * kSlice + 256 + 2 * 8 * kTeamWarps;  // two rows, histogram, scratch
+  // two staged rows, the histogram, the reduction scratch, the threads' drawn-weight scratch
+  static constexpr int kTeamWords = 2 * kSlice + 256 + 2 * 8 * kTeamWarps + kSlice;
   static constexpr size_t kBytes = static_cast<size_t>(kTeamsPerCta) * kTeamWords * 4;
 };
 
@@ -684,6 +724,7 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, VPL <= 19 ? 3 : 1) selec
   uint32_t* tw = reinterpret_cast<uint32_t*>(sm) + team * L::kTeamWords;
   uint32_t* st = tw;
   uint32_t* hist = tw + 2 * L::kSlice;
+  uint32_t* scr = hist + 256 + 2 * 8 * kTeamWarps;
   Team<kTeamWarps> tm;
   tm.red = reinterpret_cast<uint64_t*>(hist + 256);
   tm.bar_id = 1u + static_cast<uint32_t>(team);
@@ -708,7 +749,7 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, VPL <= 19 ? 3 : 1) selec
     cp_async_wait_group<1>();  // this thread's copies of the current row have landed
     tm.sync();
     if (a.discard_mass) discard_row_lines(a.mass + row * a.nK, a.nK, tm.t, 32 * kTeamWarps);
-    select_row_team<VPL, kTeamWarps>(a, row, st + buf * L::kSlice, hist, tm);
+    select_row_team<VPL, kTeamWarps>(a, row, st + buf * L::kSlice, hist, scr + tm.t * VPL, tm);
     tm.sync();  // the buffer is restaged only after every thread is done with it
     buf ^= 1;
   }
