@@ -254,22 +254,36 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
     kmax = block_max_u32(kmax, sh);
     const double mmax = static_cast<double>(__uint_as_float(kmax));
     const double c31 = mmax > 0.0 ? 2147483648.0 / mmax : 0.0;
-    for (int i = i0; i < i1; ++i) wq[i] = (flag[i] & 1) ? 0u : quant_weight(key[i], mmax, c31);
-    int n_capped = 0;
-    for (;;) {
-      uint64_t t = 0;
-      for (int i = i0; i < i1; ++i)
-        if (!(flag[i] & 3)) t += wq[i];
-      T = block_sum_u64(t, sh);
-      n_left = n_sample - n_capped;
-      uint64_t add = 0;
-      for (int i = i0; i < i1; ++i)
-        if (!(flag[i] & 3) && static_cast<uint64_t>(n_left) * wq[i] >= T) ++add;
-      add = block_sum_u64(add, sh);  // all counts are taken before any flag changes
-      if (add == 0) break;
-      for (int i = i0; i < i1; ++i)
-        if (!(flag[i] & 3) && static_cast<uint64_t>(n_left) * wq[i] >= T) flag[i] |= 2;
-      n_capped += static_cast<int>(add);
+    // the weights with their sum and maximum in one pass
+    uint64_t t0 = 0;
+    uint32_t wmax = 0;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t w = (flag[i] & 1) ? 0u : quant_weight(key[i], mmax, c31);
+      wq[i] = w;
+      t0 += w;
+      wmax = max(wmax, w);
+    }
+    T = block_sum_u64(t0, sh);
+    n_left = n_sample;
+    // capping (see the team kernel); no block is capped when even the largest
+    // weight stays below T / n_s
+    if (static_cast<uint64_t>(n_sample) * block_max_u32(wmax, sh) >= T) {
+      int n_capped = 0;
+      for (;;) {
+        uint64_t add = 0;
+        for (int i = i0; i < i1; ++i)
+          if (!(flag[i] & 3) && static_cast<uint64_t>(n_left) * wq[i] >= T) ++add;
+        add = block_sum_u64(add, sh);  // all counts are taken before any flag changes
+        if (add == 0) break;
+        for (int i = i0; i < i1; ++i)
+          if (!(flag[i] & 3) && static_cast<uint64_t>(n_left) * wq[i] >= T) flag[i] |= 2;
+        n_capped += static_cast<int>(add);
+        uint64_t t = 0;
+        for (int i = i0; i < i1; ++i)
+          if (!(flag[i] & 3)) t += wq[i];
+        T = block_sum_u64(t, sh);
+        n_left = n_sample - n_capped;
+      }
     }
     if (n_left > 0) {
       const uint32_t U = static_cast<uint32_t>(
