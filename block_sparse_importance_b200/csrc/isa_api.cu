@@ -331,7 +331,12 @@ int plan_chunk_heads(const isa_shape* s) {
   const size_t per_head = static_cast<size_t>(s->num_groups) * nblocks(s) * 4;
   size_t hc = per_head ? kPlanChunkMassBytes / per_head : 1;
   if (hc < 1) hc = 1;
-  if (hc > static_cast<size_t>(s->heads)) hc = static_cast<size_t>(s->heads);
+  const size_t H = s->heads > 0 ? static_cast<size_t>(s->heads) : 1;
+  if (hc > H) hc = H;
+  // the same number of chunks with the heads spread evenly over them, so that
+  // no chunk is a small remainder that leaves most SMs idle
+  const size_t chunks = (H + hc - 1) / hc;
+  hc = (H + chunks - 1) / chunks;
   return static_cast<int>(hc);
 }
 

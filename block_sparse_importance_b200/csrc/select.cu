@@ -149,9 +149,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelShared sh;
   const int nK = a.nK;
+  // shared memory: the keys, replaced in place by the weights of the rest
+  // once the exact set and the rest's maximum are known (nothing reads a key
+  // after that); a flag byte per block; the list of the drawn weights
   uint32_t* key = reinterpret_cast<uint32_t*>(sm);
-  uint32_t* wq = key + nK;
-  uint8_t* flag = reinterpret_cast<uint8_t*>(wq + nK);
+  uint32_t* wq = key;
+  uint8_t* flag = reinterpret_cast<uint8_t*>(key + nK);
+  uint32_t* wl = reinterpret_cast<uint32_t*>(sm + ((static_cast<size_t>(nK) * 5 + 15) & ~static_cast<size_t>(15)));
   const int tid = threadIdx.x;
   const int64_t row = blockIdx.x;
   const int g = static_cast<int>(row % a.G);
@@ -166,7 +170,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   const int i0 = min(nK, tid * E), i1 = min(nK, i0 + E);
 
   if (tid == 0) sh.bad = 0;
+  for (int i = tid; i < 256; i += kSelThreads) sh.hist[i] = 0;
   __syncthreads();
+  // the keys, with the first radix round's histogram of their top byte
   for (int i = tid; i < nK; i += kSelThreads) {
     const float v = m[i];
     uint32_t k = 0;
@@ -177,6 +183,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
     }
     key[i] = k;
     flag[i] = 0;
+    if (n_exact > 0) atomicAdd(&sh.hist[k >> 24], 1u);
   }
   __syncthreads();
   if (a.discard_mass) discard_row_lines(m, nK, tid, kSelThreads);
@@ -186,11 +193,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
     uint32_t prefix = 0, mask = 0;
     if (tid == 0) sh.remaining = n_exact;
     for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kSelThreads) sh.hist[i] = 0;
-      __syncthreads();
-      for (int i = i0; i < i1; ++i) {
-        const uint32_t k = key[i];
-        if ((k & mask) == prefix) atomicAdd(&sh.hist[(k >> shift) & 255u], 1u);
+      if (shift < 24) {
+        for (int i = tid; i < 256; i += kSelThreads) sh.hist[i] = 0;
+        __syncthreads();
+        for (int i = i0; i < i1; ++i) {
+          const uint32_t k = key[i];
+          if ((k & mask) == prefix) atomicAdd(&sh.hist[(k >> shift) & 255u], 1u);
+        }
       }
       __syncthreads();
       if (tid < 32) {
@@ -326,8 +335,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   // ---- write the plan row: exact ascending, then capped + drawn ascending.
   // The drawn blocks' log-weights are left to a second, converged pass over
   // the rest part of the row: per rest position, the drawn block's weight (0
-  // for a capped block) goes to a list over the key array, which nothing
-  // reads any more.
+  // for a capped block) goes to the list.
   int32_t* out_idx = a.idx + row * S;
   float* out_lw = a.log_w + row * S;
   const int n_rs = S - n_exact;
@@ -341,7 +349,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectLaunch a) {
   const uint64_t pre = block_scan_u64((ne << 32) | nr, sh, &tot);  // both counts < 2^32 (its barriers also
                                                                   // order every key read before the list)
   uint64_t pe = pre >> 32, pr = pre & 0xFFFFFFFFull;
-  uint32_t* wl = key;
   for (int i = i0; i < i1; ++i) {
     const uint8_t f = flag[i];
     if (f & 1) {
@@ -892,7 +899,9 @@ int launch_select(const SelectLaunch& s, cudaStream_t stream) {
   if (s.nK <= TT * 9) return launch_select_team<9>(s, stream);
   if (s.nK <= TT * 19) return launch_select_team<19>(s, stream);
   if (s.nK <= TT * 33) return launch_select_team<33>(s, stream);
-  const size_t smem = static_cast<size_t>(s.nK) * 9 + 16;
+  // keys (weights in place) and flags, then the list of the drawn weights
+  const size_t smem = ((static_cast<size_t>(s.nK) * 5 + 15) & ~static_cast<size_t>(15)) +
+                      static_cast<size_t>(s.n_exact + s.n_sample) * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel), static_cast<int>(smem));
     if (e != cudaSuccess) return static_cast<int>(e);
