@@ -785,14 +785,20 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, VPL <= 19 ? 3 : 1) selec
 //   target = ceil(p * sum q) in fp64 (the sum is below 2^45: exact),
 //   k_e = min(S, smallest k whose k largest blocks, ties to the lower block,
 //         sum to >= target).
-// The largest key t with sum_{key >= t} q >= target is found bit by bit; all
-// blocks above t are in, and of the blocks at t (equal q) the lowest
+// The largest key t with sum_{key >= t} q >= target is found byte by byte
+// from the top (a radix search whose histogram sums q instead of counting);
+// all blocks above t are in, and of the blocks at t (equal q) the lowest
 // ceil((target - sum_{key > t} q) / q_t).
 __global__ void __launch_bounds__(kSelThreads) top_p_count_kernel(const float* __restrict__ mass, int nK,
                                                                   double top_p, int S, int32_t* __restrict__ ne_rows,
                                                                   int* status) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelShared sh;
+  // per bin, the sum of q over the keys in it, as two 32-bit words (64-bit
+  // shared-memory atomics are much slower): the low word, and the number of
+  // times it wrapped
+  __shared__ uint32_t hq_lo[256], hq_hi[256];
+  __shared__ uint64_t s_above;  // sum of q over the keys above the current bin
   uint32_t* key = reinterpret_cast<uint32_t*>(sm);
   uint32_t* q = key + nK;
   const int tid = threadIdx.x;
@@ -832,12 +838,74 @@ __global__ void __launch_bounds__(kSelThreads) top_p_count_kernel(const float* _
   const uint64_t target = static_cast<uint64_t>(ceil(top_p * static_cast<double>(total)));
   int k_e = 0;
   if (target > 0) {
-    uint32_t t = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = t | (1u << bit);
-      uint64_t s = 0;
-      for (int i = i0; i < i1; ++i) s += key[i] >= cand ? q[i] : 0u;
-      if (block_sum_u64(s, sh) >= target) t = cand;
+    // byte by byte: among the keys that match the bytes found so far, the
+    // highest bin whose q-sum, with everything above it, reaches the target
+    uint32_t t = 0, mask = 0;
+    uint64_t above = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kSelThreads) {
+        hq_lo[i] = 0;
+        hq_hi[i] = 0;
+      }
+      __syncthreads();
+      {
+        // a thread's neighbouring blocks often share a bin: their q are
+        // summed locally and added once per run
+        auto add = [&](uint32_t bin, uint64_t v) {
+          const uint32_t lo = static_cast<uint32_t>(v);
+          const uint32_t old = atomicAdd(&hq_lo[bin], lo);
+          const uint32_t carry = (static_cast<uint32_t>(v >> 32)) + (old + lo < old ? 1u : 0u);
+          if (carry) atomicAdd(&hq_hi[bin], carry);
+        };
+        uint32_t run_bin = 256;
+        uint64_t run = 0;  // < E 2^31
+        for (int i = i0; i < i1; ++i) {
+          const uint32_t k = key[i], w = q[i];  // w < 2^31
+          if ((k & mask) == t && w != 0u) {
+            const uint32_t bin = (k >> shift) & 255u;
+            if (bin != run_bin) {
+              if (run_bin < 256) add(run_bin, run);
+              run_bin = bin;
+              run = 0;
+            }
+            run += w;
+          }
+        }
+        if (run_bin < 256) add(run_bin, run);
+      }
+      auto hq = [&](int i) -> uint64_t { return (static_cast<uint64_t>(hq_hi[i]) << 32) | hq_lo[i]; };
+      __syncthreads();
+      if (tid < 32) {
+        // lane l owns bins [8l, 8l+8); suffix sums from the top bin down
+        uint64_t local = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) local += hq(8 * tid + i);
+        uint64_t suf = local;  // sum of the bins owned by lanes >= tid
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint64_t x = __shfl_down_sync(0xffffffffu, suf, o);
+          if (tid + o < 32) suf += x;
+        }
+        const uint64_t need = target - above;  // > 0
+        const uint64_t higher = suf - local;   // bins of higher lanes
+        if (higher < need && suf >= need) {
+          uint64_t acc = higher;
+          for (int i = 7; i >= 0; --i) {
+            const uint64_t c = hq(8 * tid + i);
+            if (acc + c >= need) {
+              sh.sel_bin = 8 * tid + i;
+              s_above = above + acc;
+              break;
+            }
+            acc += c;
+          }
+        }
+      }
+      __syncthreads();
+      t |= sh.sel_bin << shift;
+      mask |= 255u << shift;
+      above = s_above;
+      __syncthreads();
     }
     uint64_t gt_sum = 0, gt_cnt = 0;
     for (int i = i0; i < i1; ++i) {
