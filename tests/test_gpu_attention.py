@@ -114,3 +114,26 @@ def test_host_checks_reject_bad_arguments(isa):
     bad.num_groups = 3
     with pytest.raises(isa.IsaError):
         isa.attention(q, k, v, idx, lw, bad)
+
+
+@pytest.mark.parametrize("Bk,ne,ns", [(64, 4, 7), (16, 8, 16)])
+def test_logit_jumps_match_oracle(isa, Bk, ne, ns):
+    """Plans whose later blocks carry log-weights far above the earlier ones
+    (jumps of 30, 50 and 100 nats, i.e. 43, 72 and 144 log2 units, at the last
+    or a middle plan position) and far below (-100): the running max must be
+    raised, P rescaled and O kept finite on every such path."""
+    c = Case("wan13", 2, 1200, Bk, 128, ne, ns)
+    idx, lw = c.plan()
+    lw = lw.copy()
+    S = lw.shape[-1]
+    jumps = [(S - 1, 30.0), (S - 1, 50.0), (S - 1, 100.0), (S // 2, 60.0), (S // 2, -100.0), (0, 0.0)]
+    for h in range(c.H):
+        for g in range(c.G):
+            pos, add = jumps[(h * c.G + g) % len(jumps)]
+            lw[0, h, g, pos] += add
+    q, k, v = c.cuda()
+    out, lse = isa.attention(q, k, v, torch.from_numpy(idx).cuda(), torch.from_numpy(lw).cuda(), c.layout(),
+                             want_lse=True)
+    assert isa.context().sync_status() == isa.ISA_OK
+    ref, ref_lse = c.oracle_attention(idx, lw)
+    cases.check_attention(out, ref, lse, ref_lse)
