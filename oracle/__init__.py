@@ -73,6 +73,8 @@ def _load():
             lib.ref_cluster_update.argtypes = [P, i32, i32, P, i32, P, P]
             lib.ref_cluster_update.restype = None
             lib.ref_cluster_tokens.argtypes = [P, i32, i32, i32, i32, i32, f64, P, P, P, P, P, i32]
+            lib.ref_tail_merge.argtypes = [P, i32, P, i32, i32, P, P, P, P]
+            lib.ref_tail_merge.restype = i32
             lib.ref_num_threads.restype = i32
             _lib = lib
     return _lib
@@ -180,6 +182,32 @@ def cluster_tokens(x: np.ndarray, n_clusters: int, n_iters: int, tie_rel: float 
     if st != 0:
         raise ValueError("ref_cluster_tokens: need N >= 1, 1 <= C <= N, n_iters >= 1")
     return lab, perm, off, mu, amb.astype(bool)
+
+
+def tail_merge(offsets: np.ndarray, idx: np.ndarray, k_block: int):
+    """Merged tail tiles of the permuted layout, per (batch, head).
+
+    offsets [G+1] int32 (shared by every head); idx [B, H, G, S] int32 plans.
+    Returns a list over b*H + h of (members [n, 4], slots [n, 4], ulen [n],
+    units [n, 4 S]): the tiles in the order they were opened, each with its
+    member clusters (-1 past the last), the first row of each member's slot,
+    and the union of the members' plan blocks, ascending."""
+    off = _c(offsets, np.int32)
+    idx = _c(idx, np.int32)
+    B, H, G, S = idx.shape
+    assert len(off) == G + 1
+    n_tails = int(np.count_nonzero(np.diff(off) % 128))
+    res = []
+    for bh in range(B * H):
+        mem = np.full((max(n_tails, 1), 4), -1, np.int32)
+        slo = np.full((max(n_tails, 1), 4), -1, np.int32)
+        ul = np.zeros(max(n_tails, 1), np.int32)
+        un = np.zeros((max(n_tails, 1), 4 * S), np.int32)
+        rows = idx.reshape(B * H, G, S)[bh]
+        n = _load().ref_tail_merge(_p(off), G, _p(np.ascontiguousarray(rows)), S, k_block, _p(mem), _p(slo),
+                                   _p(ul), _p(un))
+        res.append((mem[:n], slo[:n], ul[:n], un[:n]))
+    return res
 
 
 def mass_group(mu: np.ndarray, counts: np.ndarray, kbar: np.ndarray, L: np.ndarray, scale: float):

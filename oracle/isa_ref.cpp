@@ -13,6 +13,9 @@
 //         one sample per query cluster).
 //   [PH]  Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
 //         1, 2, 3" (SC'11): the Philox4x64-10 counter-based generator.
+//   [IC]  "iCATS: Fast Video Generation via Interaction-Aware Sparse Attention
+//         and Timestep-Adaptive Sparsity" (AI summary, "Approach": top-p and
+//         the merging of query-cluster tails).
 //
 // The pages give no equations; every rule marked (reading) below is the
 // plainest reading that the rest of the pages supports.
@@ -27,7 +30,10 @@
 // Token clustering (the permuted layout): brute-force nearest centroid, the
 // stable sort against a library stable argsort, the mean update against
 // numpy, the one-cluster closed form, a non-increasing objective, and the
-// recovery of well-separated generated clusters.
+// recovery of well-separated generated clusters.  Tail merging: worked
+// examples done by hand (join order, Hamming-nearest choice, ties), the closed
+// forms for identical and disjoint plans, and the schedule's rules on random
+// inputs (partition of the tails, slots, unions, no merge that costs work).
 // Parity unpinned (fixed by reading, checked only GPU-vs-oracle): the
 // k-means initialisation, the ln(L_b) term of the mass, tie-breaks, canonical
 // plan order, the 2^31 weight quantisation, the clustering's round count.
@@ -36,6 +42,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <iterator>
 #include <vector>
 
 #ifdef _OPENMP
@@ -720,6 +727,99 @@ int32_t ref_cluster_tokens(const uint16_t* x, int32_t BH, int32_t N, int32_t d, 
     ambiguous[bh] = any;
   }
   return 0;
+}
+
+// ---------------------------------------------------------------------------
+// Tail merging of the permuted layout.  [IC] "Approach": the tail blocks of
+// query clusters are merged with Hamming-nearest compatible clusters, to cut
+// the padding of their last tiles.  Readings:
+//  * the tail of cluster g is its last t_g = n_g mod 128 rows (all of it when
+//    n_g < 128; no tail when t_g = 0); in a merged 128-row tile it takes a slot
+//    of ceil(t_g / 8) * 8 rows, members packed from row 0 in the order they
+//    joined;
+//  * tails are taken in order of decreasing t_g, ties to the lower g;
+//  * a tail is compatible with an open tile when its slot fits in the rows
+//    left, the tile has fewer than 4 members, and the union U of the members'
+//    plan blocks, with the tail's plan P added, needs fewer KV tiles of
+//    128 / Bk blocks than U and P apart: ceil(|U u P| / b) < ceil(|U| / b) +
+//    ceil(|P| / b);
+//  * it joins the compatible tile whose union is Hamming-nearest to P
+//    (|U xor P| smallest, ties to the tile opened first), else opens a tile;
+//  * every row keeps its own cluster's plan and log-weights: the merged tile
+//    runs the blocks of U in ascending order, and a block outside a row's plan
+//    is masked for that row, so each row's attention is unchanged.
+// One (batch, head): off [G+1], idx [G][S] (that head's plan rows).  Outputs,
+// one entry per tile in the order the tiles were opened: members[t][4] (the
+// clusters, -1 past the last), slots[t][4] (first row of each member's slot),
+// ulen[t] and units[t][4 S] (U ascending).  Returns the number of tiles.
+int32_t ref_tail_merge(const int32_t* off, int32_t G, const int32_t* idx, int32_t S, int32_t Bk,
+                       int32_t* members, int32_t* slots, int32_t* ulen, int32_t* units) {
+  const int32_t b = 128 / Bk;
+  auto tiles_of = [&](int64_t n) { return (n + b - 1) / b; };
+  struct Tail {
+    int32_t g, t;
+  };
+  std::vector<Tail> tails;
+  for (int32_t g = 0; g < G; ++g) {
+    const int32_t t = (off[g + 1] - off[g]) % 128;
+    if (t > 0) tails.push_back({g, t});
+  }
+  std::stable_sort(tails.begin(), tails.end(), [](const Tail& x, const Tail& y) { return x.t > y.t; });
+  struct Tile {
+    int32_t rows, n;
+    int32_t g[4], slot[4];
+    std::vector<int32_t> u;  // ascending
+  };
+  std::vector<Tile> tiles;
+  for (const Tail& tl : tails) {
+    std::vector<int32_t> p(idx + static_cast<int64_t>(tl.g) * S, idx + static_cast<int64_t>(tl.g + 1) * S);
+    std::sort(p.begin(), p.end());
+    const int32_t rows = (tl.t + 7) / 8 * 8;
+    int32_t best = -1;
+    int64_t best_h = 0;
+    std::vector<int32_t> best_u;
+    for (size_t i = 0; i < tiles.size(); ++i) {
+      const Tile& tt = tiles[i];
+      if (tt.rows + rows > 128 || tt.n >= 4) continue;
+      std::vector<int32_t> un;
+      std::set_union(tt.u.begin(), tt.u.end(), p.begin(), p.end(), std::back_inserter(un));
+      if (tiles_of(static_cast<int64_t>(un.size())) >=
+          tiles_of(static_cast<int64_t>(tt.u.size())) + tiles_of(static_cast<int64_t>(p.size())))
+        continue;
+      const int64_t inter = static_cast<int64_t>(tt.u.size() + p.size() - un.size());
+      const int64_t ham = static_cast<int64_t>(tt.u.size() + p.size()) - 2 * inter;
+      if (best < 0 || ham < best_h) {
+        best = static_cast<int32_t>(i);
+        best_h = ham;
+        best_u = un;
+      }
+    }
+    if (best < 0) {
+      Tile tt;
+      tt.rows = rows;
+      tt.n = 1;
+      tt.g[0] = tl.g;
+      tt.slot[0] = 0;
+      tt.u = p;
+      tiles.push_back(tt);
+    } else {
+      Tile& tt = tiles[best];
+      tt.g[tt.n] = tl.g;
+      tt.slot[tt.n] = tt.rows;
+      ++tt.n;
+      tt.rows += rows;
+      tt.u = best_u;
+    }
+  }
+  for (size_t i = 0; i < tiles.size(); ++i) {
+    for (int32_t m = 0; m < 4; ++m) {
+      members[4 * i + m] = m < tiles[i].n ? tiles[i].g[m] : -1;
+      slots[4 * i + m] = m < tiles[i].n ? tiles[i].slot[m] : -1;
+    }
+    ulen[i] = static_cast<int32_t>(tiles[i].u.size());
+    std::copy(tiles[i].u.begin(), tiles[i].u.end(), units + static_cast<int64_t>(i) * 4 * S);
+  }
+  return static_cast<int32_t>(tiles.size());
 }
 
 int32_t ref_num_threads(void) {

@@ -41,7 +41,9 @@ def _compare(isa, mass, ne, ns, seed, H, G, nK, Bk=64):
                                       (200, 150, 50),
                                       # rows longer than 2048 blocks take the CTA-per-row kernel
                                       (2049, 0, 30), (3000, 40, 80), (7425, 248, 496), (5000, 4990, 5),
-                                      (4100, 100, 4000)])
+                                      (4100, 100, 4000),
+                                      # pure top-k (no sample), on both kernels
+                                      (64, 8, 0), (3000, 40, 0)])
 def test_select_bit_exact(isa, kind, nK, ne, ns):
     rng = np.random.default_rng(nK + ne)
     H, G = 2, 8
