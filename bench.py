@@ -361,6 +361,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--top-p", type=float, default=0.0,
                     help="also time isa_select_top_p (exact set by a share of the mass) on the step's mass")
+    ap.add_argument("--tail-merge", action="store_true",
+                    help="also time isa_tail_merge and isa_attention_merged on the step's plan (variable groups only)")
     ap.add_argument("--cluster", type=int, default=0,
                     help="also time the permuted layout's build: isa_cluster of Q and of K with this many clusters "
                          "(3 rounds) and the row permutations of Q, K and V")
@@ -512,6 +514,30 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         dense_ms = e0.elapsed_time(e1) / 2
+
+    # tail merging of the permuted layout on the step's plan: the schedule, and
+    # the attention over it (same outputs as the tile-by-tile pass)
+    if rank == 0 and args.tail_merge and w.variable_groups:
+        sched = isa.tail_merge(idx, lw, lay, ctx=ctx)
+        out_m = torch.empty_like(q)
+        isa.attention_merged(q, k, v, idx, lw, lay, sched, out=out_m, ctx=ctx)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        for _ in range(3):
+            isa.tail_merge(idx, lw, lay, schedule=sched, ctx=ctx)
+        e1.record(stream)
+        for _ in range(3):
+            isa.attention_merged(q, k, v, idx, lw, lay, sched, out=out_m, ctx=ctx)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        st = ctx.sync_status()
+        if st != isa.ISA_OK:
+            raise RuntimeError("device status after tail merging: %s" % isa.status_string(st))
+        tm_ms, am_ms = e0.elapsed_time(e1) / 3, e1.elapsed_time(e2) / 3
+        stages["tail_merge"] = {"merge_ms": tm_ms, "attention_merged_ms": am_ms,
+                                "attention_ms": attn_ms, "tflops_merged": flops / (am_ms * 1e-3) / 1e12,
+                                "what": "isa_tail_merge, then isa_attention_merged on the step's plan"}
+        del sched, out_m
 
     # the top-p selector on the same mass (count kernel + selector): mass read
     # twice, plan and per-row exact-set sizes written

@@ -626,6 +626,103 @@ isa_status isa_dense_attention(isa_context* ctx, const isa_shape* shape, const v
                       static_cast<cudaStream_t>(stream));
 }
 
+size_t isa_tail_merge_workspace_bytes(const isa_shape* s, int32_t n_sel) {
+  if (!s || s->batch < 1 || s->heads < 1 || s->num_groups < 1 || s->seq_len < 1 || s->k_block < 1 || n_sel < 1)
+    return 0;
+  return merge_carve(s->batch * s->heads, s->seq_len, s->num_groups, n_sel, nblocks(s)).total;
+}
+
+isa_status isa_tail_merge(isa_context* ctx, const isa_shape* shape, const int32_t* idx, const float* log_w,
+                          int32_t n_sel, void* schedule, size_t schedule_bytes, void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  if (!shape->q_offsets) return fail(ctx, ISA_ERR_INVALID_ARG, "tail merging needs q_offsets (the permuted layout)");
+  ISA_TRY(check_ptr(ctx, idx, "idx", 4));
+  ISA_TRY(check_ptr(ctx, log_w, "log_w", 4));
+  if (n_sel < 1) return fail(ctx, ISA_ERR_INVALID_ARG, "n_sel must be >= 1");
+  const size_t need = isa_tail_merge_workspace_bytes(shape, n_sel);
+  if (!schedule || schedule_bytes < need)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "schedule %zu bytes < %zu needed", schedule_bytes, need);
+  if (!aligned(schedule, 256)) return fail(ctx, ISA_ERR_INVALID_ARG, "schedule not 256-byte aligned");
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  const int BH = shape->batch * shape->heads;
+  const MergeCarve c = merge_carve(BH, shape->seq_len, shape->num_groups, n_sel, nblocks(shape));
+  char* w = static_cast<char*>(schedule);
+  MergeLaunch m{};
+  m.BH = BH;
+  m.N = shape->seq_len;
+  m.G = shape->num_groups;
+  m.S = n_sel;
+  m.Bk = shape->k_block;
+  m.nK = nblocks(shape);
+  m.W = (m.nK + 31) / 32;
+  m.q_offsets = shape->q_offsets;
+  m.idx = idx;
+  m.log_w = log_w;
+  m.bins = reinterpret_cast<MergeBin*>(w + c.bins);
+  m.counts = reinterpret_cast<int32_t*>(w + c.counts);
+  m.order = reinterpret_cast<int32_t*>(w + c.order);
+  m.state = reinterpret_cast<uint32_t*>(w + c.state);
+  m.prefix = reinterpret_cast<int32_t*>(w + c.prefix);
+  m.unions = reinterpret_cast<int32_t*>(w + c.unions);
+  m.tables = reinterpret_cast<float*>(w + c.tables);
+  m.items = reinterpret_cast<WorkItem*>(w + c.items);
+  m.item_count = reinterpret_cast<int32_t*>(w + c.item_count);
+  m.status = ctx->d_status;
+  return cuda_status(ctx, launch_tail_merge(m, static_cast<cudaStream_t>(stream)), "isa_tail_merge");
+}
+
+isa_status isa_attention_merged(isa_context* ctx, const isa_shape* shape, const void* q, const void* k, const void* v,
+                                const int32_t* idx, const float* log_w, int32_t n_sel, const void* schedule,
+                                size_t schedule_bytes, void* out, float* lse, void* stream) {
+  ISA_TRY(check_shape(ctx, shape));
+  if (!shape->q_offsets) return fail(ctx, ISA_ERR_INVALID_ARG, "merged attention needs q_offsets");
+  ISA_TRY(check_ptr(ctx, q, "q", 16));
+  ISA_TRY(check_ptr(ctx, k, "k", 16));
+  ISA_TRY(check_ptr(ctx, v, "v", 16));
+  ISA_TRY(check_ptr(ctx, out, "out", 16));
+  ISA_TRY(check_ptr(ctx, idx, "idx", 4));
+  ISA_TRY(check_ptr(ctx, log_w, "log_w", 4));
+  if (lse && !aligned(lse, 4)) return fail(ctx, ISA_ERR_INVALID_ARG, "lse not 4-byte aligned");
+  if (n_sel < 1) return fail(ctx, ISA_ERR_INVALID_ARG, "n_sel must be >= 1");
+  const size_t need = isa_tail_merge_workspace_bytes(shape, n_sel);
+  if (!schedule || schedule_bytes < need)
+    return fail(ctx, ISA_ERR_INVALID_ARG, "schedule %zu bytes < %zu needed", schedule_bytes, need);
+  if (!aligned(schedule, 256)) return fail(ctx, ISA_ERR_INVALID_ARG, "schedule not 256-byte aligned");
+  DeviceGuard g(ctx->device);
+  if (!g.ok()) return fail(ctx, ISA_ERR_CUDA, "cannot select device %d", ctx->device);
+  const MergeCarve c =
+      merge_carve(shape->batch * shape->heads, shape->seq_len, shape->num_groups, n_sel, nblocks(shape));
+  const char* w = static_cast<const char*>(schedule);
+  AttnLaunch l{};
+  l.B = shape->batch;
+  l.H = shape->heads;
+  l.N = shape->seq_len;
+  l.D = shape->head_dim;
+  l.G = shape->num_groups;
+  l.S = n_sel;
+  l.Bk = shape->k_block;
+  l.q_block = shape->q_block;
+  l.mode = kAttnMerged;
+  l.q_offsets = shape->q_offsets;
+  l.idx = idx;
+  l.log_w = log_w;
+  l.out = out;
+  l.lse = lse;
+  l.scale = shape->scale;
+  l.status = ctx->d_status;
+  l.num_sms = ctx->num_sms;
+  l.wait_timeout_ns = ctx->wait_timeout_ns;
+  l.stall = ctx->stall_attention;
+  l.items = reinterpret_cast<const WorkItem*>(w + c.items);
+  l.item_count = reinterpret_cast<const int32_t*>(w + c.item_count);
+  l.bins = reinterpret_cast<const MergeBin*>(w + c.bins);
+  l.unions = reinterpret_cast<const int32_t*>(w + c.unions);
+  l.tables = reinterpret_cast<const float*>(w + c.tables);
+  return cuda_status(ctx, launch_attention_merged(l, q, k, v, static_cast<cudaStream_t>(stream)),
+                     "isa_attention_merged");
+}
+
 size_t isa_plan_workspace_bytes(const isa_shape* s, const isa_params* p) {
   if (!s || !p || p->n_clusters < 1 || s->heads < 1 || s->num_groups < 1 || s->k_block < 1) return 0;
   return plan_bytes(s, p);

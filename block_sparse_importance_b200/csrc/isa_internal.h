@@ -21,11 +21,60 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 // record of what has been set is kept under a mutex.
 cudaError_t ensure_smem_attr(const void* func, int bytes);
 
+// ---------------------------------------------------------- tail merging
+// One tile of cluster tails (1..4 members) of one (batch, head), and the
+// attention's work items, as isa_tail_merge lays them out in its workspace.
+struct MergeBin {
+  int32_t n;     // members
+  int32_t rows;  // rows taken by the members' 8-row slots
+  int32_t ulen;  // blocks in the union of the members' plans
+  int32_t uoff;  // first union entry in the head's union pool (tiles of 2+ members)
+  int32_t toff;  // first entry of the [n][ulen] log-weight table in the head's pool
+  int32_t pad[3];
+  int32_t g[4];     // member clusters (-1 past the last)
+  int32_t slot[4];  // first tile row of each member
+};
+struct WorkItem {
+  int32_t bh;
+  int32_t g;  // >= 0: rows [row0, row0 + nrows) of cluster g on its plan row; < 0: tile -1 - g of head bh
+  int32_t row0, nrows;
+};
+struct MergeLaunch {
+  int BH, N, G, S, Bk, nK, W;  // W = 32-bit words of an nK-bit mask
+  const int32_t* q_offsets;    // device [G+1]
+  const int32_t* idx;          // [BH, G, S]
+  const float* log_w;          // [BH, G, S]
+  MergeBin* bins;              // [BH][G]
+  int32_t* counts;             // [BH][2]: tiles of tails, merged tiles among them
+  int32_t* order;              // [BH][G] scratch: the tails in schedule order
+  uint32_t* state;             // [BH][merge_state_words] scratch, when not in shared memory
+  int32_t* prefix;             // [BH][8][W] scratch: per-warp word prefixes
+  int32_t* unions;             // [BH][G S]: union lists, ascending
+  float* tables;               // [BH][4 G S]: log-weights per member and union position
+  WorkItem* items;             // [BH (N / 128 + G)]
+  int32_t* item_count;
+  int state_in_smem;
+  int* status;
+};
+// the greedy's state per (b, h), in 32-bit words: rows, members and union
+// size of every tile, two plan masks and the tiles' union masks
+__host__ __device__ inline size_t merge_state_words(int G, int W) {
+  return 3 * static_cast<size_t>(G) + 2 * static_cast<size_t>(W) + static_cast<size_t>(G) * W;
+}
+// byte offsets of the parts of the workspace
+struct MergeCarve {
+  size_t bins, counts, order, state, prefix, unions, tables, items, item_count, total;
+};
+MergeCarve merge_carve(int BH, int N, int G, int S, int nK);
+constexpr size_t kMergeSmemState = 160 * 1024;  // the greedy's state up to this size stays in shared memory
+int launch_tail_merge(const MergeLaunch& m, cudaStream_t stream);
+
 // ------------------------------------------------------------- attention
 enum AttnMode : int {
   kAttnGroups = 0,  // uniform query groups of <= 128 rows: one tile per group
   kAttnList = 1,    // tile list built on the device (clusters or groups > 128 rows)
-  kAttnDense = 2    // all keys, no plan
+  kAttnDense = 2,   // all keys, no plan
+  kAttnMerged = 3   // work items of isa_tail_merge: cluster tiles and merged tail tiles
 };
 
 struct AttnLaunch {
@@ -42,9 +91,17 @@ struct AttnLaunch {
   int num_sms;
   uint64_t wait_timeout_ns;  // per-wait limit of the bounded pipeline waits
   int stall;                 // test hook: the MMA warp waits on a barrier nothing arrives at
+  // kAttnMerged: the schedule of isa_tail_merge
+  const WorkItem* items;
+  const int32_t* item_count;
+  const MergeBin* bins;   // [B H][G]
+  const int32_t* unions;  // [B H][G S]
+  const float* tables;    // [B H][4 G S]
 };
 
 size_t attn_list_workspace_bytes(int N, int G);
+// kAttnMerged (attn_merged.cu): the schedule of isa_tail_merge.
+int launch_attention_merged(const AttnLaunch& a, const void* q, const void* k, const void* v, cudaStream_t stream);
 // Builds tensor maps for q/k/v and launches.  Returns a cudaError_t value or
 // -1 if a tensor map could not be encoded.
 int launch_attention(const AttnLaunch& a, const void* q, const void* k, const void* v,

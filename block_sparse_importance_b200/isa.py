@@ -79,6 +79,10 @@ def lib():
             L.isa_attention_workspace_bytes.restype = _sz
             L.isa_attention.argtypes = [_P, S, _P, _P, _P, _P, _P, _i32, _P, _P, _P, _sz, _P]
             L.isa_dense_attention.argtypes = [_P, S, _P, _P, _P, _P, _P, _P]
+            L.isa_tail_merge_workspace_bytes.argtypes = [S, _i32]
+            L.isa_tail_merge_workspace_bytes.restype = _sz
+            L.isa_tail_merge.argtypes = [_P, S, _P, _P, _i32, _P, _sz, _P]
+            L.isa_attention_merged.argtypes = [_P, S, _P, _P, _P, _P, _P, _i32, _P, _sz, _P, _P, _P]
             L.isa_plan_workspace_bytes.argtypes = [S, Pp]
             L.isa_plan_workspace_bytes.restype = _sz
             L.isa_plan.argtypes = [_P, S, Pp, _P, _P, _P, _P, _P, _sz, _P]
@@ -383,6 +387,44 @@ def attention(q, k, v, idx, log_w, lay: Layout, out=None, lse=None, workspace=No
     st = lib().isa_attention(ctx.handle, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(log_w),
                              int(idx.shape[-1]), _ptr(out), _ptr(lse), _ptr(workspace), nb, _stream(stream))
     ctx.check(st, "isa_attention")
+    return (out, lse) if want_lse else out
+
+
+def tail_merge_workspace_bytes(lay: Layout, n_sel: int) -> int:
+    return int(lib().isa_tail_merge_workspace_bytes(ctypes.byref(lay.c()), int(n_sel)))
+
+
+def tail_merge(idx, log_w, lay: Layout, schedule=None, ctx: Optional[Context] = None, stream=None):
+    """isa_tail_merge: the merged-tail schedule of a plan (permuted layout);
+    returns the schedule buffer (uint8) for attention_merged."""
+    ctx = ctx or context(idx.device.index or 0)
+    _dev(idx, torch.int32, "idx")
+    _dev(log_w, torch.float32, "log_w")
+    n_sel = int(idx.shape[-1])
+    nb = tail_merge_workspace_bytes(lay, n_sel)
+    schedule = _workspace(nb, idx.device, schedule)
+    st = lib().isa_tail_merge(ctx.handle, ctypes.byref(lay.c()), _ptr(idx), _ptr(log_w), n_sel, _ptr(schedule), nb,
+                              _stream(stream))
+    ctx.check(st, "isa_tail_merge")
+    return schedule
+
+
+def attention_merged(q, k, v, idx, log_w, lay: Layout, schedule, out=None, lse=None, ctx: Optional[Context] = None,
+                     stream=None, want_lse: bool = False):
+    """isa_attention_merged: the sparse pass over the schedule of tail_merge."""
+    ctx = ctx or context(q.device.index or 0)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, torch.bfloat16, n)
+    _dev(idx, torch.int32, "idx")
+    _dev(log_w, torch.float32, "log_w")
+    out = out if out is not None else torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = _empty(q.shape[:3], torch.float32, q.device)
+    n_sel = int(idx.shape[-1])
+    nb = schedule.numel() * schedule.element_size()
+    st = lib().isa_attention_merged(ctx.handle, ctypes.byref(lay.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
+                                    _ptr(log_w), n_sel, _ptr(schedule), nb, _ptr(out), _ptr(lse), _stream(stream))
+    ctx.check(st, "isa_attention_merged")
     return (out, lse) if want_lse else out
 
 

@@ -279,6 +279,48 @@ ISA_API isa_status isa_attention(isa_context* ctx, const isa_shape* shape, const
                          void* stream);
 
 /* ---------------------------------------------------------------------------
+ * isa_tail_merge -- tail merging for the permuted layout ("iCATS: Fast Video
+ * Generation via Interaction-Aware Sparse Attention and Timestep-Adaptive
+ * Sparsity", AI summary, "Approach": the tail blocks of query clusters are
+ * merged with Hamming-nearest compatible clusters, to cut the padding of their
+ * last tiles).  shape->q_offsets must be set.  From the plan idx, log_w
+ * ([B,H,G,n_sel], the blocks of a row distinct, as isa_select writes them) it
+ * builds per (b, h) the schedule isa_attention_merged runs:
+ *   - the tail of cluster g is its last t = n_g mod 128 rows (none when 0); it
+ *     takes a slot of ceil(t / 32) * 32 rows of a 128-row tile (whole
+ *     quarters: each softmax warp's 32 rows share one plan);
+ *   - tails are taken by decreasing t (ties: lower g).  A tail joins an open
+ *     tile when its slot fits, the tile has fewer than 4 members, and the
+ *     union U of the members' plans with the tail's plan P added needs fewer
+ *     KV tiles of 128 / k_block blocks than U and P apart; of those tiles it
+ *     joins the one whose U is nearest to P in Hamming distance (ties: the
+ *     tile opened first); otherwise it opens a tile;
+ *   - a merged tile runs the blocks of U in ascending order, and every row
+ *     keeps its own cluster's plan and log-weights (a block outside it is
+ *     masked for that row), so each output row equals isa_attention's up to
+ *     rounding.
+ * schedule: device buffer of isa_tail_merge_workspace_bytes(shape, n_sel)
+ * bytes, 256-byte aligned, owned by the caller.  It holds the schedule until
+ * it is overwritten: a plan reused across calls reuses its schedule.  An idx
+ * entry outside [0, nK) sets ISA_ERR_DEVICE_CHECK.
+ * ------------------------------------------------------------------------- */
+ISA_API size_t isa_tail_merge_workspace_bytes(const isa_shape* shape, int32_t n_sel);
+ISA_API isa_status isa_tail_merge(isa_context* ctx, const isa_shape* shape, const int32_t* idx, const float* log_w,
+                                  int32_t n_sel, void* schedule, size_t schedule_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * isa_attention_merged -- isa_attention over the schedule isa_tail_merge
+ * built from the same plan and shape: the full 128-row tiles of every cluster
+ * on the cluster's plan, then the tail tiles, a merged one on the union of its
+ * members' plans with per-row log-weights.  q, k, v, idx, log_w, n_sel, out and
+ * lse as in isa_attention (every row of N written once); schedule read only.
+ * ------------------------------------------------------------------------- */
+ISA_API isa_status isa_attention_merged(isa_context* ctx, const isa_shape* shape, const void* q, const void* k,
+                                        const void* v, const int32_t* idx, const float* log_w, int32_t n_sel,
+                                        const void* schedule, size_t schedule_bytes, void* out, float* lse,
+                                        void* stream);
+
+/* ---------------------------------------------------------------------------
  * isa_dense_attention -- the 100%-density limit: softmax(scale Q K^T) V over
  * all keys ("AB-Attention", problem statement: full attention weighs every
  * query against every key, which the sparse pass estimates; with every block

@@ -735,8 +735,9 @@ int32_t ref_cluster_tokens(const uint16_t* x, int32_t BH, int32_t N, int32_t d, 
 // the padding of their last tiles.  Readings:
 //  * the tail of cluster g is its last t_g = n_g mod 128 rows (all of it when
 //    n_g < 128; no tail when t_g = 0); in a merged 128-row tile it takes a slot
-//    of ceil(t_g / 8) * 8 rows, members packed from row 0 in the order they
-//    joined;
+//    of ceil(t_g / 32) * 32 rows (whole quarters of the tile, so that the
+//    rows a tile's softmax handles together share one plan), members packed
+//    from row 0 in the order they joined;
 //  * tails are taken in order of decreasing t_g, ties to the lower g;
 //  * a tail is compatible with an open tile when its slot fits in the rows
 //    left, the tile has fewer than 4 members, and the union U of the members'
@@ -774,7 +775,7 @@ int32_t ref_tail_merge(const int32_t* off, int32_t G, const int32_t* idx, int32_
   for (const Tail& tl : tails) {
     std::vector<int32_t> p(idx + static_cast<int64_t>(tl.g) * S, idx + static_cast<int64_t>(tl.g + 1) * S);
     std::sort(p.begin(), p.end());
-    const int32_t rows = (tl.t + 7) / 8 * 8;
+    const int32_t rows = (tl.t + 31) / 32 * 32;
     int32_t best = -1;
     int64_t best_h = 0;
     std::vector<int32_t> best_u;
