@@ -131,3 +131,28 @@ def test_merge_host_checks(isa):
     idx, lw = c.plan()
     with pytest.raises(isa.IsaError):
         isa.tail_merge(torch.from_numpy(idx).cuda(), torch.from_numpy(lw).cuda(), c.layout())
+
+
+def test_schedule_with_state_in_global_memory(isa):
+    """About 1000 clusters of 8..30 rows over 1250 key blocks: the greedy's masks
+    (G x 40 words) no longer fit in shared memory and live in the workspace."""
+    N, Bk = 20000, 16
+    off = cases.random_offsets(N, 8, 30, seed=11)
+    c = Case("wan13", 1, N, Bk, 128, 4, 8, offsets=off, seed=11)
+    G, W = c.G, (c.nK + 31) // 32
+    assert (3 * G + 2 * W + G * W) * 4 > 160 * 1024
+    idx, lw = c.plan()
+    q, k, v = c.cuda()
+    idx_d, lw_d = torch.from_numpy(idx).cuda(), torch.from_numpy(lw).cuda()
+    lay = c.layout()
+    sched = isa.tail_merge(idx_d, lw_d, lay)
+    assert isa.context().sync_status() == isa.ISA_OK
+    got = _read_schedule(sched, c.H, N, G, idx.shape[-1], c.nK)
+    mem, slo, ul, un = oracle.tail_merge(c.offsets, idx, Bk)[0]
+    assert [t[0] for t in got[0]] == mem.tolist()
+    assert [t[1] for t in got[0]] == slo.tolist()
+    assert [t[2] for t in got[0]] == ul.tolist()
+    out, lse = isa.attention_merged(q, k, v, idx_d, lw_d, lay, sched, want_lse=True)
+    assert isa.context().sync_status() == isa.ISA_OK
+    ref_out, ref_lse = c.oracle_attention()
+    cases.check_attention(out, ref_out, lse, ref_lse)
