@@ -669,6 +669,11 @@ isa_status isa_tail_merge(isa_context* ctx, const isa_shape* shape, const int32_
   m.items = reinterpret_cast<WorkItem*>(w + c.items);
   m.item_count = reinterpret_cast<int32_t*>(w + c.item_count);
   m.status = ctx->d_status;
+  {
+    // the attention's grid for these items (isa_attention_merged launches the same)
+    const long long pairs = (static_cast<long long>(BH) * (m.G + m.N / 128) + 1) / 2;
+    m.grid = static_cast<int>(pairs < ctx->num_sms ? pairs : ctx->num_sms);
+  }
   return cuda_status(ctx, launch_tail_merge(m, static_cast<cudaStream_t>(stream)), "isa_tail_merge");
 }
 

@@ -54,6 +54,7 @@ struct MergeLaunch {
   WorkItem* items;             // [BH (N / 128 + G)]
   int32_t* item_count;
   int state_in_smem;
+  int grid;  // CTAs of the attention that runs the items (merged tiles are spread over them)
   int* status;
 };
 // the greedy's state per (b, h), in 32-bit words: rows, members and union

@@ -354,6 +354,78 @@ __global__ void __launch_bounds__(kMergeThreads) merge_items_kernel(MergeLaunch 
   if (bh == 0 && tid == 0) *m.item_count = multi_all + m.BH * F + single_all;
 }
 
+// The merged tiles of all heads, spread over the attention's persistent
+// CTAs.  The grid takes the item pairs round-robin (pair p runs on CTA
+// p mod grid), and merged tiles differ in length, so the pairs are ordered by
+// length, longest first, and dealt to the CTAs in alternating direction, one
+// round of `grid` pairs after another (the last, partial round in plain
+// order); each pair holds two tiles of about the same length.  One CTA sorts
+// (length, position) keys in shared memory (bitonic); more merged tiles than
+// it holds keep the per-head order.
+constexpr int kBalanceThreads = 1024;
+constexpr int kBalanceMax = 8192;
+constexpr size_t kBalanceSmem = static_cast<size_t>(kBalanceMax) * (8 + sizeof(WorkItem));
+__global__ void __launch_bounds__(kBalanceThreads) merge_balance_kernel(MergeLaunch m) {
+  extern __shared__ __align__(16) unsigned long long key[];  // [kBalanceMax], then the items
+  WorkItem* stash = reinterpret_cast<WorkItem*>(key + kBalanceMax);
+  __shared__ int s_n;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    int n = 0;
+    for (int h = 0; h < m.BH; ++h) n += m.counts[2 * h + 1];
+    s_n = n;
+  }
+  __syncthreads();
+  const int n = s_n;
+  if (n < 3 || n > kBalanceMax || m.grid < 2) return;
+  const int b = kTileRowsM / m.Bk;
+  int pow2 = 1;
+  while (pow2 < n) pow2 <<= 1;
+  for (int i = tid; i < pow2; i += kBalanceThreads) {
+    if (i < n) {
+      const WorkItem it = m.items[i];
+      stash[i] = it;
+      const int ulen = m.bins[static_cast<int64_t>(it.bh) * m.G + (-1 - it.g)].ulen;
+      const unsigned T = static_cast<unsigned>((ulen + b - 1) / b);
+      key[i] = (static_cast<unsigned long long>(0xFFFFFFFFu - T) << 32) | static_cast<unsigned>(i);
+    } else {
+      key[i] = ~0ull;  // sorts last
+    }
+  }
+  __syncthreads();
+  for (int size = 2; size <= pow2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < pow2; i += kBalanceThreads) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const unsigned long long a = key[i], c = key[j];
+          if ((a > c) == up) {
+            key[i] = c;
+            key[j] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // an odd last (shortest) tile stays last, paired with the first item after
+  // the merged ones
+  const int grid = m.grid;
+  const int n2 = n & ~1, pairs = n2 / 2;
+  const int full_rounds = pairs / grid;
+  for (int i = tid; i < n; i += kBalanceThreads) {
+    int pos = i;
+    if (i < n2) {
+      const int pr = i >> 1, r = pr / grid;
+      int c = pr - r * grid;
+      if ((r & 1) && r < full_rounds) c = grid - 1 - c;
+      pos = 2 * (r * grid + c) + (i & 1);
+    }
+    m.items[pos] = stash[static_cast<int>(key[i] & 0xFFFFFFFFu)];
+  }
+}
+
 }  // namespace
 
 MergeCarve merge_carve(int BH, int N, int G, int S, int nK) {
@@ -397,6 +469,11 @@ int launch_tail_merge(const MergeLaunch& m, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return static_cast<int>(e);
   merge_items_kernel<<<m.BH, kMergeThreads, 0, stream>>>(l);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return static_cast<int>(e);
+  e = ensure_smem_attr(reinterpret_cast<const void*>(merge_balance_kernel), static_cast<int>(kBalanceSmem));
+  if (e != cudaSuccess) return static_cast<int>(e);
+  merge_balance_kernel<<<1, kBalanceThreads, kBalanceSmem, stream>>>(l);
   return static_cast<int>(cudaGetLastError());
 }
 
