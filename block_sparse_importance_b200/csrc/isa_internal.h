@@ -26,7 +26,7 @@ cudaError_t ensure_smem_attr(const void* func, int bytes);
 // attention's work items, as isa_tail_merge lays them out in its workspace.
 struct MergeBin {
   int32_t n;     // members
-  int32_t rows;  // rows taken by the members' 8-row slots
+  int32_t rows;  // rows taken by the members' 32-row slots
   int32_t ulen;  // blocks in the union of the members' plans
   int32_t uoff;  // first union entry in the head's union pool (tiles of 2+ members)
   int32_t toff;  // first entry of the [n][ulen] log-weight table in the head's pool
