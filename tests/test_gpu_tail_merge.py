@@ -156,3 +156,75 @@ def test_schedule_with_state_in_global_memory(isa):
     assert isa.context().sync_status() == isa.ISA_OK
     ref_out, ref_lse = c.oracle_attention()
     cases.check_attention(out, ref_out, lse, ref_lse)
+
+
+def test_full_layer_varclust(isa):
+    """The permuted layout at its full size (40 heads, 75 600 rows in 600
+    clusters, as the benchmark's tail-merge run): the oracle's plans of the
+    first and last head are placed in the layer's plan, isa_tail_merge runs on
+    the whole layer, and for those heads the schedule equals the oracle's bit
+    for bit and the merged attention of sampled clusters (members of merged
+    tiles and clusters left alone) matches the oracle."""
+    from block_sparse_importance_b200 import workloads as wl
+    w = wl.preset("varclust")
+    inp = wl.make_inputs(w, "cuda")
+    q, k, v = inp.q, inp.k, inp.v
+    B, H, N, d = q.shape
+    off = inp.offsets
+    lay = isa.layout_for(q, w.k_block, w.q_block, q_offsets=torch.from_numpy(off).cuda(), scale=w.scale)
+    G, nK, S = lay.num_groups, lay.n_key_blocks, w.n_select
+    mass = isa.score(q, k, lay, w.n_clusters, w.n_iters)
+    idx, lw = isa.select(mass, lay, w.n_exact, w.n_sample, w.seed)
+    assert isa.context().sync_status() == isa.ISA_OK
+
+    heads = [0, H - 1]
+    qb = wl.bf16_bits(q[:, heads])
+    kb = wl.bf16_bits(k[:, heads])
+    vb = wl.bf16_bits(v[:, heads])
+    m_ref, _, _, _ = oracle.score(qb, kb, off, w.k_block, w.n_clusters, w.n_iters, w.scale)
+    idx_ref, lw_ref, _ = oracle.select(m_ref.astype(np.float32), w.n_exact, w.n_sample, w.seed)
+    for j, hh in enumerate(heads):
+        idx[:, hh] = torch.from_numpy(idx_ref[:, j]).cuda()
+        lw[:, hh] = torch.from_numpy(lw_ref[:, j]).cuda()
+
+    sched = isa.tail_merge(idx, lw, lay)
+    assert isa.context().sync_status() == isa.ISA_OK
+    got = _read_schedule(sched, H, N, G, S, nK)
+    ref = oracle.tail_merge(off, idx_ref, w.k_block)
+    rng = np.random.default_rng(5)
+    sample = []
+    for j, hh in enumerate(heads):
+        mem, slo, ul, un = ref[j]
+        tiles = got[hh]
+        assert len(tiles) == len(mem)
+        n_multi = 0
+        for t, (gm, gs, gl, gu) in enumerate(tiles):
+            assert gm == mem[t].tolist()
+            assert gs == slo[t].tolist()
+            assert gl == ul[t]
+            if gm[1] >= 0:
+                n_multi += 1
+                assert gu == un[t, :ul[t]].tolist()
+        assert n_multi > 50
+        merged = sorted({g for gm, _, _, _ in tiles if gm[1] >= 0 for g in gm if g >= 0})
+        alone = sorted(set(range(G)) - set(merged))
+        pick = list(rng.choice(merged, 24, replace=False)) + list(rng.choice(alone, 8, replace=False))
+        sample += [(0, j, int(g)) for g in sorted(pick)]
+
+    out, lse = isa.attention_merged(q, k, v, idx, lw, lay, sched, want_lse=True)
+    assert isa.context().sync_status() == isa.ISA_OK
+    assert torch.isfinite(out.float()).all()
+    res = oracle.attention(qb, kb, vb, off, w.k_block, idx_ref, lw_ref, w.scale, sample)
+    o_all = out[0].float().cpu().numpy()
+    l_all = lse[0].cpu().numpy()
+    g_o, r_o, g_l, r_l = [], [], [], []
+    for (_, j, g), (o, l) in zip(sample, res):
+        g_o.append(o_all[heads[j], off[g]:off[g + 1]])
+        r_o.append(o)
+        g_l.append(l_all[heads[j], off[g]:off[g + 1]])
+        r_l.append(l)
+    g_o = np.concatenate(g_o).astype(np.float64)
+    r_o = np.concatenate(r_o)
+    assert cases.rel_l2(g_o, r_o) <= cases.ATTN_REL_L2
+    assert np.abs(g_o - r_o).max() <= cases.ATTN_MAX_ABS
+    assert np.abs(np.concatenate(g_l) - np.concatenate(r_l)).max() < 2e-2
