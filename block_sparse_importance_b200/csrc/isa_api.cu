@@ -201,6 +201,8 @@ isa_status do_score(isa_context* ctx, const isa_shape* s, const void* q, const v
   l.centroids = centroids ? centroids : reinterpret_cast<float*>(w);
   w += round_up(BH * s->num_groups * C * s->head_dim * 4);
   l.counts = counts ? counts : reinterpret_cast<int32_t*>(w);
+  w += round_up(BH * s->num_groups * C * 4);
+  l.kb_next = reinterpret_cast<uint32_t*>(w);
   l.status = ctx->d_status;
   l.num_sms = ctx->num_sms;
   return cuda_status(ctx, launch_score(l, st), "isa_score");

@@ -142,6 +142,7 @@ struct ScoreLaunch {
   int32_t* counts;    // [B,H,G,C]
   uint16_t* kbar_hi;  // [B,H,nK,D] bf16 scratch: key-block means, high part
   uint16_t* kbar_lo;  // [B,H,nK,D] bf16 scratch: key-block means, low part
+  uint32_t* kb_next;  // scratch: the next key block to take (key means beside the k-means)
   int* status;
   int num_sms;
 };

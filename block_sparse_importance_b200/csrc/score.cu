@@ -6,9 +6,13 @@
 // a weight equal to its size, and the representatives score small key blocks
 // without reordering tokens.  Key blocks are summarised by their means.
 //
-// Three kernels:
+// Kernels:
 //   key_means_kernel  kbar_b = mean of the valid rows of key block b, stored
 //                     as a bf16 hi + lo pair;
+//   kmeans_tc_kernel  (d = 128, groups of at most 128 rows) the k-means on
+//                     tcgen05, one group per set of four warps; with C <= 8
+//                     it also computes the key means in extra warps, in
+//                     place of key_means_kernel;
 //   kmeans_warp_kernel  per (batch*head, group), one warp: Lloyd's
 //                     k-means, centroids initialised at rows floor(c n / C),
 //                     `iters` rounds of nearest-centroid assignment (squared
@@ -39,15 +43,13 @@ __device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float(
 // ------------------------------------------------------------ key means
 // kbar_b = mean of the valid rows of key block b, written as a bf16 hi + lo
 // pair (hi = bf16(kbar), lo = bf16(kbar - hi)) for the tensor-core mass product.
+// One warp, key block b of (batch*head) bh; lane l sums dimensions
+// PER l .. PER l + PER - 1 over the block's rows in order.
 template <int D>
-__global__ void __launch_bounds__(kScoreThreads) key_means_kernel(const uint16_t* __restrict__ k, int N, int Bk,
-                                                                  int nK, uint16_t* __restrict__ kbar_hi,
-                                                                  uint16_t* __restrict__ kbar_lo) {
+__device__ __forceinline__ void key_mean_block(const uint16_t* __restrict__ k, int N, int Bk, int nK, int64_t bh,
+                                               int b, int lane, uint16_t* __restrict__ kbar_hi,
+                                               uint16_t* __restrict__ kbar_lo) {
   using namespace isa_dev;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.x * (kScoreThreads / 32) + warp;
-  const int64_t bh = blockIdx.y;
-  if (b >= nK) return;
   constexpr int PER = D / 32;
   const int r0 = b * Bk, r1 = min(N, r0 + Bk);
   float acc[PER];
@@ -76,6 +78,34 @@ __global__ void __launch_bounds__(kScoreThreads) key_means_kernel(const uint16_t
     const uint16_t hi = bf16_bits_rn(m);
     kbar_hi[o + i] = hi;
     kbar_lo[o + i] = bf16_bits_rn(m - bf16_bits_to_f(hi));
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads) key_means_kernel(const uint16_t* __restrict__ k, int N, int Bk,
+                                                                  int nK, uint16_t* __restrict__ kbar_hi,
+                                                                  uint16_t* __restrict__ kbar_lo) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x * (kScoreThreads / 32) + warp;
+  if (b >= nK) return;
+  key_mean_block<D>(k, N, Bk, nK, blockIdx.y, b, lane, kbar_hi, kbar_lo);
+}
+
+// The key blocks a fused k-means launch left (see kmeans_tc_kernel): each warp
+// takes one block at a time from *kb_next, until all BH nK are taken.
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads) key_means_rest_kernel(const uint16_t* __restrict__ k, int N,
+                                                                       int Bk, int nK, int n_blk,
+                                                                       uint16_t* __restrict__ kbar_hi,
+                                                                       uint16_t* __restrict__ kbar_lo,
+                                                                       uint32_t* __restrict__ kb_next) {
+  const int lane = threadIdx.x & 31;
+  for (;;) {
+    int b = 0;
+    if (lane == 0) b = static_cast<int>(atomicAdd(kb_next, 1u));
+    b = __shfl_sync(0xffffffffu, b, 0);
+    if (b >= n_blk) return;
+    key_mean_block<D>(k, N, Bk, nK, b / nK, b % nK, lane, kbar_hi, kbar_lo);
   }
 }
 
@@ -376,9 +406,21 @@ __global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16
 // of the no-swizzle MN-major layout: 8 consecutive N entries of one K index
 // per 16 bytes, so each thread stores whole vectors.
 // Warp 4 kKtSets is the TMA producer.  Every wait is bounded.
+// With C' = 8 the kernel also computes key means (FUSE): kKbWarps more warps
+// stream K, which the k-means leaves most of HBM's bandwidth free for,
+// through their own small cp.async rings in the shared memory the k-means
+// does not use.  They take key blocks from a counter in global memory and
+// stop taking more once the CTA's k-means sets are done; key_means_rest_kernel
+// then takes the blocks left.  Both write kbar exactly as key_means_kernel
+// does (the same lane-to-dimension map and the same order of the sums).
 constexpr int kKtSets = 4;
 constexpr int kKtSlots = 5;
 constexpr int kKtThreads = (4 * kKtSets + 1) * 32;
+constexpr int kKbWarps = 4;    // key-mean warps of the fused kernel
+constexpr int kKbStages = 3;   // ring chunks per key-mean warp
+constexpr int kKbRows = 8;     // key rows per chunk
+constexpr uint32_t kKbChunk = kKbRows * 128 * 2;
+constexpr int kKtThreadsFused = kKtThreads + kKbWarps * 32;
 
 template <int CP>
 struct KtLayout {
@@ -400,6 +442,12 @@ struct KtLayout {
   static constexpr int kXFull = 0, kXEmpty = kKtSlots, kMmaDone = 2 * kKtSlots, kNumBars = 2 * kKtSlots + kKtSets;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // TMEM address, abort flag; released[] at +16
   static constexpr uint32_t kAlloc = kMisc + 16 + 4 * kKtSlots + 1024;
+  // fused kernel: the count of k-means sets done, the key-mean warps' chunk
+  // descriptors [kKbWarps][kKbStages] (block, offset << 8 | rows), their rings
+  static constexpr uint32_t kKb = (kMisc + 16 + 4 * kKtSlots + 15) & ~15u;
+  static constexpr uint32_t kKbDesc = kKb + 16;
+  static constexpr uint32_t kKbRing = (kKbDesc + kKbWarps * kKbStages * 8 + 15) & ~15u;
+  static constexpr uint32_t kAllocFused = kKbRing + kKbWarps * kKbStages * kKbChunk + 1024;
 };
 
 // Byte offset of element (row r, column c) in a K-major 128-byte-swizzled
@@ -432,11 +480,13 @@ __device__ __forceinline__ float warp_sum_scatter(float (&v)[CP], int lane, int&
   return r;
 }
 
-template <int CP>
-__global__ void __launch_bounds__(kKtThreads, 1)
+template <int CP, bool FUSE>
+__global__ void __launch_bounds__(FUSE ? kKtThreadsFused : kKtThreads, 1)
     kmeans_tc_kernel(const __grid_constant__ CUtensorMap tm_q, int BH, int N, int G, int q_block,
                      const int32_t* __restrict__ off, int C, int iters, float* __restrict__ centroids,
-                     int32_t* __restrict__ counts, uint64_t timeout_ns, int* status) {
+                     int32_t* __restrict__ counts, uint64_t timeout_ns, int* status,
+                     const uint16_t* __restrict__ kmat, int Bk, int nK, uint16_t* __restrict__ kbar_hi,
+                     uint16_t* __restrict__ kbar_lo, uint32_t* __restrict__ kb_next) {
   using namespace isa_dev;
   using L = KtLayout<CP>;
   constexpr int D = 128;
@@ -465,10 +515,15 @@ __global__ void __launch_bounds__(kKtThreads, 1)
     fence_mbar_init();
   }
   // one-hot slots of clusters >= C stay zero, and the counts start at zero
-  for (int i = tid; i < static_cast<int>(kKtSets * L::kOhBytes / 16); i += kKtThreads)
-    reinterpret_cast<uint4*>(smem + L::kOh)[i] = make_uint4(0u, 0u, 0u, 0u);
-  for (int i = tid; i < static_cast<int>(kKtSets * L::kRedBytes / 4); i += kKtThreads)
-    reinterpret_cast<uint32_t*>(smem + L::kRed)[i] = 0u;
+  if constexpr (FUSE) {
+    if (tid == 0) *reinterpret_cast<volatile int*>(smem + L::kKb) = 0;
+  }
+  if (tid < kKtThreads) {
+    for (int i = tid; i < static_cast<int>(kKtSets * L::kOhBytes / 16); i += kKtThreads)
+      reinterpret_cast<uint4*>(smem + L::kOh)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid; i < static_cast<int>(kKtSets * L::kRedBytes / 4); i += kKtThreads)
+      reinterpret_cast<uint32_t*>(smem + L::kRed)[i] = 0u;
+  }
   fence_proxy_async_smem();
   if (warp == kProducer) {
     tmem_alloc(smem_addr(tmem_slot), 256);
@@ -533,7 +588,7 @@ __global__ void __launch_bounds__(kKtThreads, 1)
         }
       }
     }
-  } else {
+  } else if (warp < kProducer) {
     // ------------------------------------------------------- k-means sets
     const int s = warp >> 2, q4 = warp & 3;
     const int t = q4 * 32 + lane;  // TMEM lane: the X row (assign) or the dimension (update)
@@ -774,6 +829,12 @@ __global__ void __launch_bounds__(kKtThreads, 1)
         if (c < C) centroids[(o * C + c) * D + t] = mu[c];
       if (t < C) counts[o * C + t] = static_cast<int32_t>(my_count);
     }
+    if constexpr (FUSE) {
+      // this set takes no more groups: the key-mean warps stop taking blocks
+      // once every set of the CTA is here
+      __syncwarp();
+      if (q4 == 0 && lane == 0) atomicAdd(reinterpret_cast<int*>(smem + L::kKb), 1);
+    }
     if (pending && q4 == q_mma) {
       // a batch whose wait gave up may still be running: let it finish before
       // the tensor memory is freed
@@ -781,6 +842,104 @@ __global__ void __launch_bounds__(kKtThreads, 1)
       while (!mbar_try_wait(bar(L::kMmaDone + s), mma_waits & 1u))
         if (global_timer_ns() - t0 > 200000000ull) break;
     }
+  } else if constexpr (FUSE) {
+    // ------------------------------------------------- key means (fused)
+    // The warp takes kb_run key blocks at a time from *kb_next and streams
+    // their rows through its ring in chunks of at most kKbRows rows, a chunk
+    // never crossing a block (each lane copies up to four 16-byte pieces);
+    // the chunk's (block, offset, rows) goes to the warp's descriptor slot.
+    // Lane l sums dimensions 4l .. 4l + 3 of every row in order, and the
+    // block's last chunk writes its mean.  No block is taken once all of the
+    // CTA's k-means sets are done; the stream then ends with the chunks in
+    // flight.
+    const int kw = warp - kProducer - 1;
+    const int n_blk = BH * nK;
+    const int kb_run = Bk >= 64 ? 1 : 64 / Bk;
+    volatile int* sets_done = reinterpret_cast<volatile int*>(smem + L::kKb);
+    volatile int* desc = reinterpret_cast<volatile int*>(smem + L::kKbDesc) + 2 * kw * kKbStages;
+    const uint32_t ring = base + L::kKbRing + static_cast<uint32_t>(kw) * (kKbStages * kKbChunk);
+    const uint8_t* ring_p = smem + L::kKbRing + static_cast<uint32_t>(kw) * (kKbStages * kKbChunk);
+    auto rows_of_block = [&](int b) -> int {
+      const int kb = b % nK;
+      return min(N, (kb + 1) * Bk) - kb * Bk;
+    };
+    // issue side (warp-uniform): the block being cut into chunks, the end of
+    // the run it belongs to, the next chunk's row offset in it
+    int cur_b = 0, run_end = 0, cur_off = 0;
+    bool more = true;
+    auto issue = [&](int c) {
+      int b = -1, o = 0, rows = 0;
+      if (more && cur_b >= run_end) {
+        int r0 = n_blk;
+        if (lane == 0 && *sets_done < kKtSets) r0 = static_cast<int>(atomicAdd(kb_next, static_cast<uint32_t>(kb_run)));
+        r0 = __shfl_sync(0xffffffffu, r0, 0);
+        if (r0 >= n_blk) {
+          more = false;
+        } else {
+          cur_b = r0;
+          run_end = min(n_blk, r0 + kb_run);
+          cur_off = 0;
+        }
+      }
+      if (more) {
+        b = cur_b;
+        o = cur_off;
+        const int rb = rows_of_block(b);
+        rows = min(kKbRows, rb - o);
+        cur_off += rows;
+        if (cur_off >= rb) {
+          ++cur_b;
+          cur_off = 0;
+        }
+        const int bh = b / nK, kb = b - bh * nK;
+        const uint16_t* src = kmat + (static_cast<int64_t>(bh) * N + static_cast<int64_t>(kb) * Bk + o) * 128;
+        const uint32_t dst = ring + static_cast<uint32_t>(c % kKbStages) * kKbChunk;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int piece = lane + 32 * j;  // 16-byte piece of the chunk; row piece / 16
+          if ((piece >> 4) < rows) cp_async16(dst + piece * 16, src + piece * 8);
+        }
+      }
+      if (lane == 0) {
+        desc[2 * (c % kKbStages)] = b;
+        desc[2 * (c % kKbStages) + 1] = (o << 8) | rows;
+      }
+      cp_async_commit();  // an empty group past the end keeps the count regular
+    };
+#pragma unroll
+    for (int c = 0; c < kKbStages - 1; ++c) issue(c);
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int c = 0;; ++c) {
+      issue(c + kKbStages - 1);
+      cp_async_wait_group<kKbStages - 1>();  // this lane's pieces of chunk c have landed
+      __syncwarp();                           // and the other lanes' too, and its descriptor
+      const int d_b = desc[2 * (c % kKbStages)], d_or = desc[2 * (c % kKbStages) + 1];
+      if (d_b < 0) break;
+      const int rows = d_or & 255, o = d_or >> 8;
+      const uint8_t* chunk = ring_p + static_cast<uint32_t>(c % kKbStages) * kKbChunk;
+      for (int i = 0; i < rows; ++i) {
+        const uint2 v = *reinterpret_cast<const uint2*>(chunk + i * 256 + lane * 8);
+        acc[0] += bf16_to_f(v.x & 0xFFFF);
+        acc[1] += bf16_to_f(v.x >> 16);
+        acc[2] += bf16_to_f(v.y & 0xFFFF);
+        acc[3] += bf16_to_f(v.y >> 16);
+      }
+      const int rb = rows_of_block(d_b);
+      if (o + rows == rb) {
+        const float inv = 1.0f / static_cast<float>(rb);
+        const int64_t out = static_cast<int64_t>(d_b) * 128 + lane * 4;  // (bh nK + b) d
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float m = acc[e] * inv;
+          const uint16_t hi = bf16_bits_rn(m);
+          kbar_hi[out + e] = hi;
+          kbar_lo[out + e] = bf16_bits_rn(m - bf16_bits_to_f(hi));
+          acc[e] = 0.0f;
+        }
+      }
+      __syncwarp();  // every lane has read the chunk and its descriptor before the slot is reused
+    }
+    cp_async_wait_group<0>();
   }
   tc_fence_before();
   __syncthreads();
@@ -1181,26 +1340,35 @@ int launch_mass_any(const ScoreLaunch& s, int nK, int BH, cudaStream_t stream) {
   }
 }
 
-// The tensor-core k-means over the groups of at most 128 rows (d = 128, C <= 16).
-cudaError_t launch_kmeans_tc(const ScoreLaunch& s, int BH, cudaStream_t stream) {
+static_assert(KtLayout<8>::kAllocFused <= 227 * 1024 && KtLayout<8>::kAlloc < KtLayout<8>::kAllocFused,
+              "the fused k-means must fit the shared memory of one CTA");
+static_assert(KtLayout<16>::kAlloc <= 227 * 1024 && KtLayout<16>::kAlloc < KtLayout<16>::kAllocFused,
+              "C' = 16 runs without the key-mean warps");
+
+// The tensor-core k-means over the groups of at most 128 rows (d = 128, C <= 16);
+// with C <= 8 the same launch also writes the key means (kbar hi / lo).
+cudaError_t launch_kmeans_tc(const ScoreLaunch& s, int BH, int nK, cudaStream_t stream) {
   CUtensorMap tq;
   if (!make_bf16_map(&tq, s.q, BH, s.N, 128, 128)) return cudaErrorInvalidValue;
   const long long items = static_cast<long long>(BH) * s.G;
   const int grid = static_cast<int>(items < s.num_sms ? items : s.num_sms);
+  const uint16_t* kmat = static_cast<const uint16_t*>(s.k);
   if (s.C <= 8) {
     using L = KtLayout<8>;
-    const cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kmeans_tc_kernel<8>), L::kAlloc);
+    const cudaError_t e =
+        ensure_smem_attr(reinterpret_cast<const void*>(kmeans_tc_kernel<8, true>), static_cast<int>(L::kAllocFused));
     if (e != cudaSuccess) return e;
-    kmeans_tc_kernel<8><<<grid, kKtThreads, L::kAlloc, stream>>>(tq, BH, s.N, s.G, s.q_block, s.q_offsets, s.C,
-                                                                 s.iters, s.centroids, s.counts, kWaitTimeoutNs,
-                                                                 s.status);
+    kmeans_tc_kernel<8, true><<<grid, kKtThreadsFused, L::kAllocFused, stream>>>(
+        tq, BH, s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids, s.counts, kWaitTimeoutNs, s.status,
+        kmat, s.Bk, nK, s.kbar_hi, s.kbar_lo, s.kb_next);
   } else {
     using L = KtLayout<16>;
-    const cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kmeans_tc_kernel<16>), L::kAlloc);
+    const cudaError_t e =
+        ensure_smem_attr(reinterpret_cast<const void*>(kmeans_tc_kernel<16, false>), static_cast<int>(L::kAlloc));
     if (e != cudaSuccess) return e;
-    kmeans_tc_kernel<16><<<grid, kKtThreads, L::kAlloc, stream>>>(tq, BH, s.N, s.G, s.q_block, s.q_offsets, s.C,
-                                                                  s.iters, s.centroids, s.counts, kWaitTimeoutNs,
-                                                                  s.status);
+    kmeans_tc_kernel<16, false><<<grid, kKtThreads, L::kAlloc, stream>>>(
+        tq, BH, s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids, s.counts, kWaitTimeoutNs, s.status,
+        kmat, s.Bk, nK, s.kbar_hi, s.kbar_lo, s.kb_next);
   }
   return cudaGetLastError();
 }
@@ -1209,16 +1377,31 @@ template <int D>
 int launch_score_d(const ScoreLaunch& s, cudaStream_t stream) {
   const int BH = s.B * s.H;
   const int nK = (s.N + s.Bk - 1) / s.Bk;
-  key_means_kernel<D><<<dim3((nK + 7) / 8, BH), kScoreThreads, 0, stream>>>(static_cast<const uint16_t*>(s.k), s.N,
-                                                                            s.Bk, nK, s.kbar_hi, s.kbar_lo);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaSuccess;
+  // the key means have their own launch unless the tensor-core k-means
+  // (d = 128, C <= 8) computes them alongside, taking blocks from *kb_next;
+  // key_means_rest_kernel then takes the blocks left
+  const bool fused = D == 128 && s.C <= 8;
+  if (fused) {
+    e = cudaMemsetAsync(s.kb_next, 0, sizeof(uint32_t), stream);
+  } else {
+    key_means_kernel<D><<<dim3((nK + 7) / 8, BH), kScoreThreads, 0, stream>>>(static_cast<const uint16_t*>(s.k),
+                                                                              s.N, s.Bk, nK, s.kbar_hi, s.kbar_lo);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return static_cast<int>(e);
   // groups of at most 128 rows (every group of the uniform layouts) take the
   // tensor-core k-means when d = 128 and C <= 16; the rest, the per-warp one
   int warp_min_rows = 0;
   if (D == 128 && s.C <= 16) {
-    e = launch_kmeans_tc(s, BH, stream);
+    e = launch_kmeans_tc(s, BH, nK, stream);
     if (e != cudaSuccess) return static_cast<int>(e);
+    if (fused) {
+      key_means_rest_kernel<D><<<s.num_sms * 8, kScoreThreads, 0, stream>>>(
+          static_cast<const uint16_t*>(s.k), s.N, s.Bk, nK, BH * nK, s.kbar_hi, s.kbar_lo, s.kb_next);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return static_cast<int>(e);
+    }
     warp_min_rows = 128;
     if (!s.q_offsets && s.q_block <= 128) return launch_mass_any<D>(s, nK, BH, stream);
   }
@@ -1263,7 +1446,7 @@ size_t score_workspace_bytes(int B, int H, int N, int D, int G, int Bk, int C) {
   const size_t BH = static_cast<size_t>(B) * H;
   const size_t nK = (static_cast<size_t>(N) + Bk - 1) / Bk;
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  return up(BH * nK * D * 4) + up(BH * G * C * D * 4) + up(BH * G * C * 4);
+  return up(BH * nK * D * 4) + up(BH * G * C * D * 4) + up(BH * G * C * 4) + up(sizeof(uint32_t));
 }
 
 int launch_score(const ScoreLaunch& s, cudaStream_t stream) {

@@ -40,7 +40,7 @@ def test_workspace_sizes(L):
     nk = 1182
     want = (40 * nk * 128 * 4) + (40 * 591 * 8 * 128 * 4) + (40 * 591 * 8 * 4)
     got = isa.score_workspace_bytes(lay, 8)
-    assert want <= got <= want + 3 * 256
+    assert want + 4 <= got <= want + 4 * 256                       # + the key-block counter
     assert isa.attention_workspace_bytes(lay) == 0                 # uniform groups need no scratch
     lay.q_block = 200
     lay.num_groups = -(-75600 // 200)
