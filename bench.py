@@ -521,7 +521,7 @@ def main():
         sched = isa.tail_merge(idx, lw, lay, ctx=ctx)
         out_m = torch.empty_like(q)
         isa.attention_merged(q, k, v, idx, lw, lay, sched, out=out_m, ctx=ctx)
-        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0, e1, e2, e3 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
         e0.record(stream)
         for _ in range(3):
             isa.tail_merge(idx, lw, lay, schedule=sched, ctx=ctx)
@@ -529,14 +529,20 @@ def main():
         for _ in range(3):
             isa.attention_merged(q, k, v, idx, lw, lay, sched, out=out_m, ctx=ctx)
         e2.record(stream)
+        # the tile-by-tile pass timed the same way, right after
+        for _ in range(3):
+            isa.attention(q, k, v, idx, lw, lay, out=out_m, workspace=aws, ctx=ctx)
+        e3.record(stream)
         torch.cuda.synchronize()
         st = ctx.sync_status()
         if st != isa.ISA_OK:
             raise RuntimeError("device status after tail merging: %s" % isa.status_string(st))
-        tm_ms, am_ms = e0.elapsed_time(e1) / 3, e1.elapsed_time(e2) / 3
+        tm_ms, am_ms, at_ms = e0.elapsed_time(e1) / 3, e1.elapsed_time(e2) / 3, e2.elapsed_time(e3) / 3
         stages["tail_merge"] = {"merge_ms": tm_ms, "attention_merged_ms": am_ms,
-                                "attention_ms": attn_ms, "tflops_merged": flops / (am_ms * 1e-3) / 1e12,
-                                "what": "isa_tail_merge, then isa_attention_merged on the step's plan"}
+                                "attention_same_loop_ms": at_ms, "attention_step_ms": attn_ms,
+                                "tflops_merged": flops / (am_ms * 1e-3) / 1e12,
+                                "what": "isa_tail_merge, then isa_attention_merged on the step's plan, then "
+                                        "isa_attention timed the same way (3 back-to-back calls each)"}
         del sched, out_m
 
     # the top-p selector on the same mass (count kernel + selector): mass read
