@@ -416,8 +416,8 @@ __global__ void __launch_bounds__(kKmWarps * 32) kmeans_warp_kernel(const uint16
 constexpr int kKtSets = 4;
 constexpr int kKtSlots = 5;
 constexpr int kKtThreads = (4 * kKtSets + 1) * 32;
-constexpr int kKbWarps = 4;    // key-mean warps of the fused kernel
-constexpr int kKbStages = 3;   // ring chunks per key-mean warp
+constexpr int kKbWarps = 6;    // key-mean warps of the fused kernel
+constexpr int kKbStages = 2;   // ring chunks per key-mean warp
 constexpr int kKbRows = 8;     // key rows per chunk
 constexpr uint32_t kKbChunk = kKbRows * 128 * 2;
 constexpr int kKtThreadsFused = kKtThreads + kKbWarps * 32;
