@@ -1346,19 +1346,27 @@ static_assert(KtLayout<16>::kAlloc <= 227 * 1024 && KtLayout<16>::kAlloc < KtLay
               "C' = 16 runs without the key-mean warps");
 
 // The tensor-core k-means over the groups of at most 128 rows (d = 128, C <= 16);
-// with C <= 8 the same launch also writes the key means (kbar hi / lo).
-cudaError_t launch_kmeans_tc(const ScoreLaunch& s, int BH, int nK, cudaStream_t stream) {
+// with `fused` (C <= 8) the same launch also writes the key means (kbar hi / lo).
+cudaError_t launch_kmeans_tc(const ScoreLaunch& s, int BH, int nK, bool fused, cudaStream_t stream) {
   CUtensorMap tq;
   if (!make_bf16_map(&tq, s.q, BH, s.N, 128, 128)) return cudaErrorInvalidValue;
   const long long items = static_cast<long long>(BH) * s.G;
   const int grid = static_cast<int>(items < s.num_sms ? items : s.num_sms);
   const uint16_t* kmat = static_cast<const uint16_t*>(s.k);
-  if (s.C <= 8) {
+  if (s.C <= 8 && fused) {
     using L = KtLayout<8>;
     const cudaError_t e =
         ensure_smem_attr(reinterpret_cast<const void*>(kmeans_tc_kernel<8, true>), static_cast<int>(L::kAllocFused));
     if (e != cudaSuccess) return e;
     kmeans_tc_kernel<8, true><<<grid, kKtThreadsFused, L::kAllocFused, stream>>>(
+        tq, BH, s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids, s.counts, kWaitTimeoutNs, s.status,
+        kmat, s.Bk, nK, s.kbar_hi, s.kbar_lo, s.kb_next);
+  } else if (s.C <= 8) {
+    using L = KtLayout<8>;
+    const cudaError_t e =
+        ensure_smem_attr(reinterpret_cast<const void*>(kmeans_tc_kernel<8, false>), static_cast<int>(L::kAlloc));
+    if (e != cudaSuccess) return e;
+    kmeans_tc_kernel<8, false><<<grid, kKtThreads, L::kAlloc, stream>>>(
         tq, BH, s.N, s.G, s.q_block, s.q_offsets, s.C, s.iters, s.centroids, s.counts, kWaitTimeoutNs, s.status,
         kmat, s.Bk, nK, s.kbar_hi, s.kbar_lo, s.kb_next);
   } else {
@@ -1380,8 +1388,9 @@ int launch_score_d(const ScoreLaunch& s, cudaStream_t stream) {
   cudaError_t e = cudaSuccess;
   // the key means have their own launch unless the tensor-core k-means
   // (d = 128, C <= 8) computes them alongside, taking blocks from *kb_next;
-  // key_means_rest_kernel then takes the blocks left
-  const bool fused = D == 128 && s.C <= 8;
+  // key_means_rest_kernel then takes the blocks left (block indices are int:
+  // layers of 2^30 key blocks and more keep the separate launch)
+  const bool fused = D == 128 && s.C <= 8 && static_cast<int64_t>(BH) * nK < (int64_t{1} << 30);
   if (fused) {
     e = cudaMemsetAsync(s.kb_next, 0, sizeof(uint32_t), stream);
   } else {
@@ -1394,7 +1403,7 @@ int launch_score_d(const ScoreLaunch& s, cudaStream_t stream) {
   // tensor-core k-means when d = 128 and C <= 16; the rest, the per-warp one
   int warp_min_rows = 0;
   if (D == 128 && s.C <= 16) {
-    e = launch_kmeans_tc(s, BH, nK, stream);
+    e = launch_kmeans_tc(s, BH, nK, fused, stream);
     if (e != cudaSuccess) return static_cast<int>(e);
     if (fused) {
       key_means_rest_kernel<D><<<s.num_sms * 8, kScoreThreads, 0, stream>>>(
