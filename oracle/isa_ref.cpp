@@ -34,7 +34,9 @@
 // examples done by hand (join order, Hamming-nearest choice, ties), the closed
 // forms for identical and disjoint plans, and the schedule's rules on random
 // inputs (partition of the tails, slots, unions, no merge that costs work).
-// Parity unpinned (fixed by reading, checked only GPU-vs-oracle): the
+// Choices the pages leave open (each is a stated reading; the functions that
+// make them are pinned by the checks above, but no page value can pin the
+// choice itself, so the GPU matches the oracle on them by construction): the
 // k-means initialisation, the ln(L_b) term of the mass, tie-breaks, canonical
 // plan order, the 2^31 weight quantisation, the clustering's round count.
 
